@@ -1,0 +1,186 @@
+"""Seeded synthetic inputs for the VGG-T^3 test-time-training layer.
+
+This module holds shapes, layouts and random draws only; none of the layer's
+arithmetic lives here.  Both the float64 oracle (through the tests) and the
+CUDA path take their inputs from it.
+
+Workloads (token layout per view: ``n_special`` camera/register tokens first,
+then the ``grid_h x grid_w`` patch grid in row-major order):
+
+* VGG-T^3 paper, Sec. 3.1 "Tokenization": a 518x518 image with patch size 14
+  gives a 37x37 = 1369 patch grid; camera and register tokens are appended.
+* VGG-T^3 paper, Sec. 3.2 / App. A: per-head width 64 (VGGT width 1024 = 16 x 64),
+  SwiGLU fast-weight MLP, 1 inner step for short collections and 2 at 1k views.
+
+Distributions: Q and K rows are L2-normalised N(0,1) draws per (token, head)
+row of length d (the pages' L2 normalisation of Q and K, Sec. 3.2), then
+rounded to bfloat16; V ~ N(0,1) rounded to bfloat16; depthwise 3x3 weights
+~ N(0, 1/9); fast weights Xavier-normal with std sqrt(2 / (d + h)).
+
+Every view of every token tensor is drawn from its own generator, seeded by a
+SplitMix64 mix of (seed, tensor id, view index), so any subset or permutation
+of views reproduces the same values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Iterable, Optional, Sequence
+
+import torch
+
+__all__ = [
+    "LayerConfig", "CONFIGS", "make_inputs", "pack_theta", "unpack_theta",
+    "theta_numel", "bf16_round", "view_token_index",
+]
+
+_MASK64 = (1 << 64) - 1
+
+# tensor ids of the counter-based seeding
+_TID_K, _TID_Q, _TID_V, _TID_CONV, _TID_W1, _TID_W3, _TID_W2 = range(7)
+
+
+def _splitmix64(x: int) -> int:
+    """SplitMix64 output function (Steele, Lea, Flood, OOPSLA 2014)."""
+    x = (x + 0x9E3779B97F4A7C15) & _MASK64
+    z = x
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+    return z ^ (z >> 31)
+
+
+def _stream_seed(seed: int, tensor_id: int, view: int) -> int:
+    s = _splitmix64(seed & _MASK64)
+    s = _splitmix64(s ^ (tensor_id & _MASK64))
+    s = _splitmix64(s ^ (view & _MASK64))
+    return s & ((1 << 63) - 1)
+
+
+def _randn(shape, seed, tensor_id, view, device) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(_stream_seed(seed, tensor_id, view))
+    return torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerConfig:
+    """One workload of the TTT layer.
+
+    tokens per view = n_special + grid_h * grid_w; n = n_views * tokens per view.
+    """
+    name: str
+    n_views: int
+    grid_h: int
+    grid_w: int
+    n_special: int
+    heads: int
+    d: int
+    h: int
+    steps: int
+    lr: float
+    seed: int
+    fp32_inputs: bool = False      # the tiny case draws fp32 Q/K/V
+    heldout_views: int = 0         # frozen-theta read of extra views
+    heldout_seed: int = 0
+
+    @property
+    def tokens_per_view(self) -> int:
+        return self.n_special + self.grid_h * self.grid_w
+
+    @property
+    def n(self) -> int:
+        return self.n_views * self.tokens_per_view
+
+    def with_views(self, n_views: int) -> "LayerConfig":
+        return dataclasses.replace(self, n_views=n_views)
+
+    def flops(self) -> float:
+        """Algorithmic FLOPs of conv-free layer math: (14*steps + 6) * d * h per token and head."""
+        return float(14 * self.steps + 6) * self.d * self.h * self.n * self.heads
+
+    def dims(self) -> Dict[str, int]:
+        return dict(n_views=self.n_views, grid_h=self.grid_h, grid_w=self.grid_w,
+                    n_special=self.n_special, heads=self.heads, d=self.d, h=self.h)
+
+
+CONFIGS: Dict[str, LayerConfig] = {
+    c.name: c for c in [
+        # 2 views of an 8x8 grid, 1 head, d=16, h=32, fp32 draws, 1 step, lr 0.1, seed 0
+        LayerConfig("tiny_2v_8x8_d16_h32", 2, 8, 8, 0, 1, 16, 32, 1, 0.1, 0, fp32_inputs=True),
+        # 24 views of 37x37 + 5 special tokens (32,976 tokens), 16 heads, d=64, h=256, 1 step
+        LayerConfig("views24_37x37p5_h16_d64_h256", 24, 37, 37, 5, 16, 64, 256, 1, 0.1, 1),
+        # 100 views (137,400 tokens), 2 steps
+        LayerConfig("views100_37x37p5_h16_d64_h256", 100, 37, 37, 5, 16, 64, 256, 2, 0.1, 2),
+        # 1000 views (1,374,000 tokens), 2 steps, lr 0.05
+        LayerConfig("views1000_37x37p5_h16_d64_h256", 1000, 37, 37, 5, 16, 64, 256, 2, 0.05, 3),
+        # 2000 views, one fast-weight MLP d=1024, h=2048, 2 steps, lr 0.02, + 200 held-out views
+        LayerConfig("views2000_37x37p5_h1_d1024_h2048", 2000, 37, 37, 5, 1, 1024, 2048, 2, 0.02, 4,
+                    heldout_views=200, heldout_seed=1004),
+    ]
+}
+
+
+def bf16_round(x: torch.Tensor) -> torch.Tensor:
+    """Round to bfloat16 (round-to-nearest-even) and return float32 values."""
+    return x.to(torch.bfloat16).to(torch.float32)
+
+
+def view_token_index(cfg: LayerConfig, view: int, y: int, x: int) -> int:
+    """Token index of patch (y, x) of a view; special tokens come first in each view."""
+    return view * cfg.tokens_per_view + cfg.n_special + y * cfg.grid_w + x
+
+
+def _token_tensor(cfg, tensor_id, views, device, normalise, seed) -> torch.Tensor:
+    parts = []
+    for v in views:
+        r = _randn((cfg.tokens_per_view, cfg.heads, cfg.d), seed, tensor_id, v, device)
+        if normalise:
+            r = r / torch.linalg.vector_norm(r, dim=-1, keepdim=True)
+        parts.append(r)
+    return torch.cat(parts, 0) if parts else torch.zeros(0, cfg.heads, cfg.d, device=device)
+
+
+def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] = None,
+                heldout: bool = False) -> Dict[str, torch.Tensor]:
+    """Draw the layer's inputs.
+
+    Returns float32 tensors (values already rounded to bfloat16 unless
+    ``cfg.fp32_inputs``): Q, K, V of shape [n, heads, d]; conv_w [heads*d, 3, 3];
+    W1, W3 [heads, d, h]; W2 [heads, h, d].  ``views`` selects (and orders) the
+    views drawn; ``heldout`` draws the held-out query views instead (Q only).
+    """
+    if views is None:
+        views = range(cfg.heldout_views if heldout else cfg.n_views)
+    views = list(views)
+    seed = cfg.heldout_seed if heldout else cfg.seed
+    out: Dict[str, torch.Tensor] = {}
+    rnd = (lambda t: t) if cfg.fp32_inputs else bf16_round
+    out["Q"] = rnd(_token_tensor(cfg, _TID_Q, views, device, True, seed))
+    if heldout:
+        return out
+    out["K"] = rnd(_token_tensor(cfg, _TID_K, views, device, True, seed))
+    out["V"] = rnd(_token_tensor(cfg, _TID_V, views, device, False, seed))
+    C = cfg.heads * cfg.d
+    out["conv_w"] = _randn((C, 3, 3), seed, _TID_CONV, 0, device) * (1.0 / 3.0)
+    std = math.sqrt(2.0 / (cfg.d + cfg.h))
+    out["W1"] = _randn((cfg.heads, cfg.d, cfg.h), seed, _TID_W1, 0, device) * std
+    out["W3"] = _randn((cfg.heads, cfg.d, cfg.h), seed, _TID_W3, 0, device) * std
+    out["W2"] = _randn((cfg.heads, cfg.h, cfg.d), seed, _TID_W2, 0, device) * std
+    return out
+
+
+def theta_numel(heads: int, d: int, h: int) -> int:
+    return 3 * heads * d * h
+
+
+def pack_theta(W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor) -> torch.Tensor:
+    """Flat float32 fast-weight buffer [W1: H*d*h | W3: H*d*h | W2: H*h*d], row-major."""
+    return torch.cat([W1.reshape(-1), W3.reshape(-1), W2.reshape(-1)]).to(torch.float32).contiguous()
+
+
+def unpack_theta(theta: torch.Tensor, heads: int, d: int, h: int):
+    """Inverse of :func:`pack_theta`; returns (W1, W3, W2) views."""
+    s = heads * d * h
+    t = theta.reshape(-1)
+    return (t[:s].reshape(heads, d, h), t[s:2 * s].reshape(heads, d, h),
+            t[2 * s:3 * s].reshape(heads, h, d))
