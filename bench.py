@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the VGG-T^3 TTT layer on B200.
+
+One step = one ``ttt_layer`` call over the whole workload: ShortConv2D of V,
+`steps` SGD write steps (forward residual, backward partials, reduce+update)
+and the read of Q.  Default workload: 1000 views x (37x37 + 5) tokens
+(1,374,000 tokens), 16 heads, d=64, h=256, 2 steps, lr 0.05, bf16 operands.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs an independent replica of the
+workload (its own scene; the layer has no cross-scene exchange), so the
+scaling is weak and value = all ranks' tokens / max-over-ranks time.
+``--impl reference`` times the float64 CPU oracle on bounded samples of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TTT layer tokens/s (write 2 steps + read) at 1000 views; % BF16 TC & HBM peak"
+DEFAULT_CONFIG = "views1000_37x37p5_h16_d64_h256"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_sample(cfg, n_views_sample: int, head: int = 0) -> float:
+    """Seconds of the float64 oracle on `n_views_sample` views x 1 head of the workload."""
+    import numpy as np  # noqa: F401
+    from oracle import ttt_oracle as orc
+    from test_layer_reconstruction_b200 import inputs as tin
+    sub = cfg.with_views(n_views_sample)
+    inp = tin.make_inputs(sub)
+    d = cfg.d
+    ch = slice(head * d, (head + 1) * d)
+    K = inp["K"][:, head].double().numpy()
+    Q = inp["Q"][:, head].double().numpy()
+    V = inp["V"][:, head].double().numpy()
+    w = inp["conv_w"][ch].double().numpy()
+    th0 = (inp["W1"][head].double().numpy(), inp["W3"][head].double().numpy(), inp["W2"][head].double().numpy())
+    dims = orc.Dims(sub.n_views, sub.grid_h, sub.grid_w, sub.n_special)
+    t0 = time.perf_counter()
+    Vp = orc.shortconv2d(V, w, dims)
+    th, _ = orc.sgd_write(K, Vp, th0, sub.lr, sub.steps)
+    orc.read(Q, *th)
+    return time.perf_counter() - t0
+
+
+def _oracle_tokens_per_s(cfg, seconds_budget: float):
+    """Time the oracle on a bounded sample; returns (tokens/s in layer tokens, description)."""
+    t_small = _oracle_sample(cfg, 2)
+    per_view = t_small / 2
+    views = max(2, min(cfg.n_views, int(seconds_budget / max(per_view, 1e-6))))
+    t = _oracle_sample(cfg, views)
+    tokens = views * cfg.tokens_per_view
+    # one head of `heads`: a full-layer token costs `heads` times the per-head work
+    value = tokens / (t * cfg.heads)
+    desc = (f"float64 numpy oracle, 1 of {cfg.heads} heads x {views} of {cfg.n_views} views "
+            f"({tokens} tokens, {cfg.steps} steps), {t:.2f} s; tokens/s = tokens / (time * heads)")
+    return value, desc, t
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step_budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    t_small = _oracle_sample(cfg, 2)
+    views = max(2, min(cfg.n_views, int(per_step_budget / max(t_small / 2, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_sample(cfg, views)
+    times = [_oracle_sample(cfg, views) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    tokens = views * cfg.tokens_per_view
+    value = tokens / (t * cfg.heads)
+    cores = _blas_threads()
+    sample = (f"float64 numpy oracle, 1 of {cfg.heads} heads x {views} of {cfg.n_views} views "
+              f"({tokens} tokens, {cfg.steps} steps) per step; tokens/s = tokens / (time * heads)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "n_views": cfg.n_views, "tokens": cfg.n, "heads": cfg.heads, "d": cfg.d,
+                   "h": cfg.h, "steps": cfg.steps, "lr": cfg.lr},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _kernel_work(cfg):
+    """Algorithmic work of one launch of each kernel kind (bytes or FLOPs)."""
+    n, H, d, h = cfg.n, cfg.heads, cfg.d, cfg.h
+    tok = n * H * d * 2
+    return {
+        "shortconv2d": ("hbm", 2 * tok + H * d * 9 * 4),             # read V, write V'
+        "swiglu_fwd_residual": ("tensor", 6.0 * d * h * n * H),      # Z1, Z3, Y
+        "swiglu_bwd_partials": ("tensor", 8.0 * d * h * n * H),      # dA, dW1, dW3, dW2
+        "swiglu_fwd_read": ("tensor", 6.0 * d * h * n * H),
+        "pack_theta": ("hbm", 3 * H * d * h * 4 + 3 * H * 128 * math.ceil(h / 128) * d * 2),
+        "reduce_sgd": ("hbm", 0),
+    }
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from test_layer_reconstruction_b200 import build as tbuild
+    from test_layer_reconstruction_b200 import inputs as tin
+    from test_layer_reconstruction_b200 import ttt
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    tbuild.build()
+    ttt.load_library()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # Each rank draws its own replica (seed offset by rank).
+    rcfg = tin.LayerConfig(cfg.name, cfg.n_views, cfg.grid_h, cfg.grid_w, cfg.n_special, cfg.heads, cfg.d, cfg.h,
+                           cfg.steps, cfg.lr, cfg.seed + 1000 * rank)
+    inp = tin.make_inputs(rcfg, device="cuda")
+    Q = inp["Q"].to(torch.bfloat16).contiguous()
+    K = inp["K"].to(torch.bfloat16).contiguous()
+    V = inp["V"].to(torch.bfloat16).contiguous()
+    conv_w = inp["conv_w"].contiguous()
+    theta0 = tin.pack_theta(inp["W1"], inp["W3"], inp["W2"]).cuda()
+    del inp
+    torch.cuda.empty_cache()
+    theta = torch.empty_like(theta0)
+    O = torch.empty_like(Q)
+    ws = ttt.make_workspace(cfg, ttt.OP_LAYER)
+
+    def step():
+        ttt.layer(Q, K, V, conv_w, theta0, cfg.lr, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ttt.check_status(ws) != 0:
+        raise SystemExit("device status word set during warm-up")
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ttt.profile_start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = ttt.profile_stop()
+    clk = clocks.stop()
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if ttt.check_status(ws) != 0:
+        raise SystemExit("device status word set during the timed steps")
+    ms_t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    value = world * cfg.n / (ms_max / 1e3)
+
+    # per-kernel roofline from the live event timings
+    peaks = _peaks()
+    work = _kernel_work(cfg)
+    kernels = {}
+    for name, rec in prof.items():
+        if name.startswith("_") or rec["launches"] == 0:
+            continue
+        bound, amount = work[name]
+        per_launch_ms = rec["total_ms"] / rec["launches"]
+        if bound == "tensor":
+            achieved = amount / (per_launch_ms / 1e3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            unit = "TFLOP/s"
+        else:
+            achieved = amount / (per_launch_ms / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        kernels[name] = {"launches_per_step": rec["launches"] / args.steps, "ms_per_launch": per_launch_ms,
+                         "share": rec["total_ms"] / max(1e-9, sum(r["total_ms"] for k, r in prof.items()
+                                                                  if not k.startswith("_"))),
+                         "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak if peak else None}
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches_per_step"])
+    dk = kernels[dom]
+    traffic = _traffic_from_profiles(dom)
+    roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} ({'sustained bf16' if dk['bound'] == 'tensor' else 'HBM copy'})"}
+    gpu_launches = sum(r["launches"] for k, r in prof.items() if not k.startswith("_"))
+
+    # end to end through the host-buffer entry point
+    e2e = None
+    if args.e2e_steps > 0:
+        ws_h = ttt.make_workspace(cfg, ttt.OP_LAYER_HOST)
+        hq, hk, hv = (t.cpu().pin_memory() for t in (Q, K, V))
+        hw = conv_w.cpu().pin_memory()
+        ht0 = theta0.cpu().pin_memory()
+        hth = torch.empty_like(ht0).pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        h2d = 3 * hq.numel() * 2 + hw.numel() * 4 + ht0.numel() * 4
+        d2h = ho.numel() * 2 + hth.numel() * 4
+        ttt.layer_host(hq, hk, hv, hw, ht0, cfg.lr, cfg.steps, cfg, hth, ho, ws_h)
+        torch.cuda.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            ttt.layer_host(hq, hk, hv, hw, ht0, cfg.lr, cfg.steps, cfg, hth, ho, ws_h)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = f0.elapsed_time(f1) / args.e2e_steps
+        e_t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * cfg.n / (float(e_t.item()) / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "wall_s_per_step": (time.perf_counter() - t0) / args.e2e_steps}
+        del ws_h
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, _ = _oracle_tokens_per_s(cfg, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "n_views": cfg.n_views, "tokens": cfg.n, "heads": cfg.heads,
+                       "d": cfg.d, "h": cfg.h, "steps": cfg.steps, "lr": cfg.lr,
+                       "l2": "no flush: every token tensor (2.8 GB) exceeds the 126 MB L2",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": gpu_launches, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def _traffic_from_profiles(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, when one matches the current build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get(kernel)
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from test_layer_reconstruction_b200 import inputs as tin
+    cfg = tin.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,151 @@
+/*
+ * ttt.h — C ABI of the B200 (sm_100a) VGG-T^3 test-time-training layer.
+ *
+ * The layer (VGG-T$^3$: Offline Feed-Forward 3D Reconstruction at Scale,
+ * Sec. 3.4, Eq. 3 and Eq. 4) replaces global softmax attention by
+ *   1. V' = ShortConv2D(V): a depthwise 3x3 convolution of each view's patch
+ *      grid of values ("Non-Linear Spatial Mixing via ShortConv2D"; camera and
+ *      register tokens pass through, Appendix A);
+ *   2. `steps` plain gradient steps theta <- theta - lr * grad L(theta) that fit
+ *      a per-head SwiGLU fast-weight MLP T_theta(x) = (silu(x W1) * (x W3)) W2
+ *      from K to V' under L = (1/n) sum_i ||T_theta(k_i) - v'_i||^2 (Eq. 3,
+ *      "TTT MLP Architecture and Inner Optimization");
+ *   3. the read o_i = T_theta*(q_i) (Eq. 4).
+ *
+ * Layouts (row-major, n = n_views * (n_special + grid_h * grid_w)):
+ *   Q, K, V, O     bfloat16 bit patterns, [n][heads][d] (token-major; each
+ *                  view's n_special special tokens first, then its patch grid
+ *                  row by row).
+ *   conv_w         float32 [heads*d][3][3], cross-correlation taps (row, col).
+ *   theta          float32, packed [W1: heads*d*h | W3: heads*d*h | W2: heads*h*d],
+ *                  W1/W3 per head [d][h], W2 per head [h][d].
+ *
+ * Ownership and streams: the caller owns every buffer; the library allocates
+ * no memory.  Scratch lives in a caller-provided device workspace of at least
+ * ttt_workspace_bytes(dims, op) bytes, 256-byte aligned.  All device pointers
+ * must be 16-byte aligned.  Work is enqueued on `stream` (a cudaStream_t, or
+ * NULL for the legacy default stream) and returns without synchronising;
+ * inputs are never modified.  theta_out may alias theta0 (in-place update); no
+ * other buffers may overlap.  Calls sharing one workspace must not run
+ * concurrently.
+ *
+ * Errors: host-side validation happens before anything is enqueued and
+ * returns a negative ttt_status; nothing throws across the ABI.  A failed
+ * launch returns TTT_ECUDA.  Faults detected on the device (a bounded wait that
+ * ran out) are recorded in the workspace status word, which every call taking
+ * a workspace clears when it starts, and are reported by ttt_check_status as
+ * TTT_EDEVICE.
+ *
+ * Supported shapes: d in {16, 32, 64}; 1 <= h <= 256 (padded internally to a
+ * multiple of 128 with zero weights, which is exact); heads >= 1;
+ * grid_h, grid_w >= 1; 0 <= n_special; n >= 1.  Other shapes return
+ * TTT_EUNSUPPORTED.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ttt_dims {
+  int32_t n_views;    /* views (images) in the collection                     */
+  int32_t grid_h;     /* patch-grid rows per view (H/p)                       */
+  int32_t grid_w;     /* patch-grid columns per view (W/p)                    */
+  int32_t n_special;  /* special tokens per view, stored first, not convolved */
+  int32_t heads;      /* fast-weight MLPs, one per head                       */
+  int32_t d;          /* head width (MLP input and output)                    */
+  int32_t h;          /* SwiGLU hidden width                                  */
+} ttt_dims;
+
+typedef enum ttt_status {
+  TTT_OK = 0,
+  TTT_EINVAL = -1,        /* null pointer, negative size, bad op or steps      */
+  TTT_EALIGN = -2,        /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+  TTT_EUNSUPPORTED = -3,  /* shape outside the supported set                   */
+  TTT_EWORKSPACE = -4,    /* workspace smaller than ttt_workspace_bytes        */
+  TTT_ECUDA = -5,         /* a CUDA runtime/driver call or launch failed       */
+  TTT_EDEVICE = -6        /* a kernel recorded a device-side fault             */
+} ttt_status;
+
+typedef enum ttt_op {
+  TTT_OP_WRITE = 0,       /* ttt_write                                         */
+  TTT_OP_READ = 1,        /* ttt_read                                          */
+  TTT_OP_LAYER = 2,       /* ttt_layer                                         */
+  TTT_OP_LAYER_HOST = 3   /* ttt_layer_host: also holds device copies of Q,K,V,conv_w,theta,O */
+} ttt_op;
+
+/* Bytes of device workspace an op needs for these dims; 0 if dims are invalid
+ * or unsupported. */
+size_t ttt_workspace_bytes(const ttt_dims* dims, int op);
+
+/* Step 1 alone: V_out = ShortConv2D(V) (VGG-T^3 summary, "Non-Linear Spatial
+ * Mixing via ShortConv2D", Appendix A).  V, V_out: bf16 [n][heads*d];
+ * conv_w: f32 [heads*d][3][3].  FP32 accumulation, bf16 round-to-nearest-even
+ * store.  Special tokens are copied.  Needs no workspace. */
+int ttt_shortconv2d(const ttt_dims* dims, const uint16_t* V, const float* conv_w,
+                    uint16_t* V_out, void* stream);
+
+/* Write (Eq. 3): V' = ShortConv2D(V), then `steps` (>= 0) full-batch SGD steps
+ * from theta0 with learning rate lr; theta_out receives theta*.  Operands are
+ * bf16 with FP32 accumulation; theta is kept in FP32 and rounded to bf16 for
+ * the tensor cores each step. */
+int ttt_write(const ttt_dims* dims, const uint16_t* K, const uint16_t* V,
+              const float* conv_w, const float* theta0, float lr, int steps,
+              float* theta_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Read (Eq. 4): O = T_theta(Q) with frozen theta (query mode).  dims describe
+ * Q's token count through n_views/grid/n_special; only n, heads, d, h are used. */
+int ttt_read(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole layer: ttt_write on (K, V) then ttt_read of Q with theta*. */
+int ttt_layer(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+              const float* conv_w, const float* theta0, float lr, int steps,
+              float* theta_out, uint16_t* O, void* workspace, size_t workspace_bytes,
+              void* stream);
+
+/* ttt_layer on HOST buffers: copies Q, K, V, conv_w, theta0 to device copies
+ * inside the workspace (one cudaMemcpyAsync each), runs the layer, copies
+ * theta* and O back to the host buffers, all on `stream`.  Returns once the
+ * work is enqueued; the host outputs are valid after the stream
+ * synchronises.  Pinned host memory makes the copies asynchronous.
+ * Workspace: ttt_workspace_bytes(dims, TTT_OP_LAYER_HOST). */
+int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t* K_host,
+                   const uint16_t* V_host, const float* conv_w_host,
+                   const float* theta0_host, float lr, int steps, float* theta_out_host,
+                   uint16_t* O_host, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device status word of `workspace`:
+ * TTT_OK, TTT_EDEVICE if a kernel recorded a fault (the word is cleared), or
+ * TTT_ECUDA. */
+int ttt_check_status(const void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* ttt_status_str(int status);
+
+/* Per-kernel timing, for measurement only.  Between ttt_profile_start and
+ * ttt_profile_stop the library records a CUDA event before and after every
+ * kernel it launches (on the launch stream; calling threads must not overlap).
+ * ttt_profile_stop synchronises those events and fills, per kernel kind k
+ * (0 <= k < TTT_KERNEL_KINDS, named by ttt_kernel_name), the number of
+ * launches and their summed device time in milliseconds.  At most 65536
+ * launches are recorded per session; later ones are counted in `dropped`. */
+#define TTT_KERNEL_KINDS 6
+typedef struct ttt_kernel_times {
+  int32_t launches[TTT_KERNEL_KINDS];
+  float total_ms[TTT_KERNEL_KINDS];
+  int32_t dropped;
+} ttt_kernel_times;
+int ttt_profile_start(void);
+int ttt_profile_stop(ttt_kernel_times* out);
+const char* ttt_kernel_name(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H_ */

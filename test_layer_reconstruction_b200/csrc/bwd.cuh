@@ -1,0 +1,351 @@
+// bwd.cuh — gradient of the mean-squared TTT loss w.r.t. the SwiGLU fast
+// weights, as split-K partial sums over token ranges.
+//
+// For the loss L = (1/n) sum_i ||T(k_i) - v'_i||^2 (VGG-T$^3$: Offline
+// Feed-Forward 3D Reconstruction at Scale, Sec. 3.4, Eq. 3; the gradient is a
+// sum of per-token terms, Eq. 5) with residual E = T(K) - V' from the forward
+// kernel, the chain rule through T(x) = (silu(x W1) * (x W3)) W2 gives, per
+// token tile (G = (2/n) E; the 2/n is applied in the update):
+//   Z1 = K W1, Z3 = K W3, S = sigmoid(Z1)                      (recomputed)
+//   dA = E W2^T
+//   dZ1 = dA * Z3 * S * (1 + Z1 (1 - S)),  dZ3 = dA * Z1 * S,  A = Z1 S Z3
+//   dW1^T += dZ1^T K,  dW3^T += dZ3^T K,  dW2 += A^T E
+// CTA work = (head, 128-wide slice of the hidden units, contiguous range of
+// 128-token tiles); dW for the slice stays in TMEM for the whole range and is
+// written once per (head, slice) segment to a partial buffer.  The update
+// kernel sums the partials of a (head, slice) in CTA order, so the result is
+// deterministic.
+//
+// Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
+// allocator + MMA issuer, warps 2-9 two epilogue warpgroups.  Per tile the
+// slice is walked in 4 sub-chunks of 32 hidden units, each with
+//   Z  = K * [W1 | W3]_sub   (M=128 tokens, N=64, K=d)
+//   dA = E * W2_sub^T        (M=128 tokens, N=32, K=d)
+// in one of 3 TMEM slots; the epilogue writes A, dZ1, dZ3 (bf16) to shared
+// memory and the dW MMAs (M=128 hidden, N=d, K=128 tokens, both operands
+// MN-major) of tile j are issued after the sub-chunk MMAs of tile j+1.
+#pragma once
+#include "fwd.cuh"
+
+namespace ttt {
+
+struct BwdParams {
+  const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
+  const __nv_bfloat16* w2_img;   // per head: HIDP rows of D bf16 (sw-swizzled)
+  float* partials;               // [pairs][max_contrib][3][128][D] f32
+  int n, heads, tiles, slices;   // slices = HIDP / 128
+  int max_contrib;
+  unsigned int* status;
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int SW = 2 * D;
+  static constexpr uint32_t kW13 = 2u * 128 * D * 2;  // rows of one 128-wide slice
+  static constexpr uint32_t kW2 = 1u * 128 * D * 2;
+  static constexpr uint32_t kTile = 1u * kTileM * D * 2;
+  static constexpr uint32_t kBuf = 2u * kTileM * 64 * 2;  // [128 tok][128 hid] as 2 atoms of 64
+  static constexpr uint32_t off_w13 = 0;
+  static constexpr uint32_t off_w2 = off_w13 + kW13;
+  static constexpr uint32_t off_k = off_w2 + kW2;
+  static constexpr uint32_t off_e = off_k + 2 * kTile;
+  static constexpr uint32_t off_a = off_e + 2 * kTile;
+  static constexpr uint32_t off_dz1 = off_a + kBuf;
+  static constexpr uint32_t off_dz3 = off_dz1 + kBuf;
+  static constexpr uint32_t off_bar = off_dz3 + kBuf;
+  static constexpr int kNumBars = 24;
+  static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
+  static_assert(off_k % 1024 == 0 && off_e % 1024 == 0 && off_a % 1024 == 0, "1 KiB alignment");
+};
+
+enum BwdBar {
+  BB_W_FULL = 0, BB_W_EMPTY = 1, BB_KE_FULL = 2, BB_KE_EMPTY = 4, BB_SL_FULL = 6, BB_SL_EMPTY = 9,
+  BB_DZ_FULL = 12, BB_DZ_EMPTY = 13, BB_ACC_FULL = 14, BB_ACC_EMPTY = 15, BB_DONE = 16
+};
+
+// CTA that owns flattened work item i under the static partition
+// [floor(c*N/G), floor((c+1)*N/G)).
+__host__ __device__ inline long long owner_cta(long long i, long long n_items, long long grid) {
+  return ((i + 1) * grid - 1) / n_items;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_e,
+               const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int SW = L::SW;
+  constexpr uint32_t kSlot = 96;       // TMEM columns per sub-chunk slot
+  constexpr uint32_t kDw = 288;        // first dW column
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const Abort ab{abort_flag, p.status};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const long long total = static_cast<long long>(p.heads) * p.slices * p.tiles;
+  const long long it0 = total * blockIdx.x / gridDim.x;
+  const long long it1 = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[BB_W_FULL], 1);
+    mbar_init(&bars[BB_W_EMPTY], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[BB_KE_FULL + s], 1);
+      mbar_init(&bars[BB_KE_EMPTY + s], 1);
+    }
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&bars[BB_SL_FULL + s], 1);
+      mbar_init(&bars[BB_SL_EMPTY + s], 4);
+    }
+    mbar_init(&bars[BB_DZ_FULL], 8);
+    mbar_init(&bars[BB_DZ_EMPTY], 1);
+    mbar_init(&bars[BB_ACC_FULL], 1);
+    mbar_init(&bars[BB_ACC_EMPTY], 8);
+    mbar_init(&bars[BB_DONE], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_e);
+      long long cur_pair = -1;
+      uint32_t wl = 0, j = 0;
+      for (long long it = it0; it < it1; ++it, ++j) {
+        const long long pair = it / p.tiles;
+        const int tile = static_cast<int>(it % p.tiles);
+        const int head = static_cast<int>(pair / p.slices);
+        const int slice = static_cast<int>(pair % p.slices);
+        if (pair != cur_pair) {
+          if (wl > 0 && !mbar_wait(&bars[BB_W_EMPTY], (wl - 1) & 1, ab)) break;
+          mbar_arrive_expect_tx(&bars[BB_W_FULL], L::kW13 + L::kW2);
+          const size_t hidp = static_cast<size_t>(p.slices) * 128;
+          const __nv_bfloat16* w13 = p.w13_img + (static_cast<size_t>(head) * 2 * hidp + slice * 256) * D;
+          const __nv_bfloat16* w2 = p.w2_img + (static_cast<size_t>(head) * hidp + slice * 128) * D;
+          bulk_load_pieces(smem + L::off_w13, w13, L::kW13, &bars[BB_W_FULL]);
+          bulk_load_pieces(smem + L::off_w2, w2, L::kW2, &bars[BB_W_FULL]);
+          ++wl;
+          cur_pair = pair;
+        }
+        const int s = j & 1;
+        if (!mbar_wait(&bars[BB_KE_EMPTY + s], ((j >> 1) & 1) ^ 1, ab)) break;
+        mbar_arrive_expect_tx(&bars[BB_KE_FULL + s], 2 * L::kTile);
+        tma_load_2d(smem + L::off_k + s * L::kTile, &tm_k, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
+        tma_load_2d(smem + L::off_e + s * L::kTile, &tm_e, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
+      }
+      if (wl > 0) mbar_drain(&bars[BB_W_FULL], (wl - 1) & 1);
+      for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) mbar_drain(&bars[BB_KE_FULL + (jj & 1)], (jj >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdZ = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t kIdDA = idesc_bf16(128, 32, false, false);
+      constexpr uint32_t kIdW = idesc_bf16(128, D, true, true);
+      const uint32_t w13 = smem_u32(smem + L::off_w13);
+      const uint32_t w2 = smem_u32(smem + L::off_w2);
+      const uint32_t sa = smem_u32(smem + L::off_a);
+      const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
+      const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
+      long long cur_pair = -1;
+      uint32_t wl = 0, j = 0, kc = 0, seg = 0;
+      bool ok = true, pend = false, pend_first = false;
+      uint32_t pend_j = 0;
+      // dW MMAs of tile qj (stage qj % 2); `first` starts a new accumulation.
+      auto issue_dw = [&](uint32_t qj, bool first) -> bool {
+        if (!mbar_wait(&bars[BB_DZ_FULL], qj & 1, ab)) return false;
+        if (first && seg > 0 && !mbar_wait(&bars[BB_ACC_EMPTY], (seg - 1) & 1, ab)) return false;
+        tc_fence_after();
+        const int s = qj & 1;
+        const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
+        const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
+#pragma unroll
+        for (int k = 0; k < kTileM / 16; ++k) {
+          const uint32_t acc = (first && k == 0) ? 0u : 1u;
+          const uint64_t bk = smem_desc(ks + k * 16 * SW, 0, 8 * SW, SW);
+          const uint64_t be = smem_desc(es + k * 16 * SW, 0, 8 * SW, SW);
+          mma_bf16(tbase + kDw, smem_desc(sdz1 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
+          mma_bf16(tbase + kDw + D, smem_desc(sdz3 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
+          mma_bf16(tbase + kDw + 2 * D, smem_desc(sa + k * 2048, 16384, 1024, 128), be, kIdW, acc);
+        }
+        mma_commit(&bars[BB_DZ_EMPTY]);
+        mma_commit(&bars[BB_KE_EMPTY + s]);
+        return true;
+      };
+      bool seg_first = false;
+      for (long long it = it0; it < it1 && ok; ++it, ++j) {
+        const long long pair = it / p.tiles;
+        if (pair != cur_pair) {
+          if (pend) {
+            if (!(ok = issue_dw(pend_j, pend_first))) break;
+            pend = false;
+          }
+          if (cur_pair >= 0) {
+            mma_commit(&bars[BB_ACC_FULL]);   // segment done: epilogue dumps dW
+            mma_commit(&bars[BB_W_EMPTY]);
+            ++seg;
+          }
+          if (!(ok = mbar_wait(&bars[BB_W_FULL], wl & 1, ab))) break;
+          ++wl;
+          cur_pair = pair;
+          seg_first = true;
+        }
+        const int s = j & 1;
+        if (!(ok = mbar_wait(&bars[BB_KE_FULL + s], (j >> 1) & 1, ab))) break;
+        tc_fence_after();
+        const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
+        const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
+        for (int sc = 0; sc < 4; ++sc, ++kc) {
+          const uint32_t slot = kc % 3, use = kc / 3;
+          if (!(ok = mbar_wait(&bars[BB_SL_EMPTY + slot], (use & 1) ^ 1, ab))) break;
+          tc_fence_after();
+          const uint32_t tsl = tbase + slot * kSlot;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            mma_bf16(tsl, smem_desc(ks + 32 * k, 0, 8 * SW, SW), smem_desc(w13 + 64 * sc * SW + 32 * k, 0, 8 * SW, SW),
+                     kIdZ, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            mma_bf16(tsl + 64, smem_desc(es + 32 * k, 0, 8 * SW, SW), smem_desc(w2 + 32 * sc * SW + 32 * k, 0, 8 * SW, SW),
+                     kIdDA, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars[BB_SL_FULL + slot]);
+        }
+        if (!ok) break;
+        if (pend && !(ok = issue_dw(pend_j, pend_first))) break;
+        pend = true;
+        pend_j = j;
+        pend_first = seg_first;
+        seg_first = false;
+      }
+      if (ok && pend) ok = issue_dw(pend_j, pend_first);
+      if (ok && cur_pair >= 0) mma_commit(&bars[BB_ACC_FULL]);
+      mma_commit(&bars[BB_DONE]);
+      mbar_drain(&bars[BB_DONE], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int g = (warp - 2) >> 2;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;            // token row (sub-chunks), hidden row (dW dump)
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t sa = smem_u32(smem + L::off_a);
+    const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
+    const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
+    uint32_t j = 0, seg = 0;
+    long long cur_pair = -1;
+    bool ok = true;
+
+    // Write dW of the finished segment (pair) to its partial slot.
+    auto dump = [&](long long pair) -> bool {
+      if (!mbar_wait(&bars[BB_ACC_FULL], seg & 1, ab)) return false;
+      tc_fence_after();
+      const long long first_item = pair * p.tiles;
+      const long long contrib = blockIdx.x - owner_cta(first_item, total, gridDim.x);
+      float* dst = p.partials + (static_cast<size_t>(pair) * p.max_contrib + contrib) * (3u * 128u * D);
+      for (int grp = g; grp < 3 * D / 16; grp += 2) {
+        uint32_t r[16];
+        tmem_ld16(tbase + kDw + grp * 16 + lane_off, r);
+        tmem_wait_ld();
+        const int m = grp * 16 / D, col = grp * 16 % D;
+        float4* o = reinterpret_cast<float4*>(dst + (static_cast<size_t>(m) * 128 + row) * D + col);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          o[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                             __uint_as_float(r[4 * v + 3]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BB_ACC_EMPTY]);
+      ++seg;
+      return true;
+    };
+
+    for (long long it = it0; it < it1 && ok; ++it, ++j) {
+      const long long pair = it / p.tiles;
+      if (pair != cur_pair) {
+        if (cur_pair >= 0 && !(ok = dump(cur_pair))) break;
+        cur_pair = pair;
+      }
+      bool waited_buf = false;
+      for (int sc = g; sc < 4; sc += 2) {
+        const uint32_t kc = j * 4 + sc;
+        const uint32_t slot = kc % 3, use = kc / 3;
+        if (!(ok = mbar_wait(&bars[BB_SL_FULL + slot], use & 1, ab))) break;
+        tc_fence_after();
+        const uint32_t tsl = tbase + slot * kSlot + lane_off;
+        uint32_t pa[16], pz1[16], pz3[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t z1[16], z3[16], da[16];
+          tmem_ld16(tsl + half * 16, z1);
+          tmem_ld16(tsl + 32 + half * 16, z3);
+          tmem_ld16(tsl + 64 + half * 16, da);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            float av[2], d1[2], d3[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const float x1 = __uint_as_float(z1[i + t]), x3 = __uint_as_float(z3[i + t]);
+              const float dav = __uint_as_float(da[i + t]);
+              const float sg = sigmoid_fast(x1);
+              const float silu = x1 * sg;
+              const float tt = x3 * sg;
+              av[t] = silu * x3;
+              d1[t] = dav * fmaf(tt * x1, 1.0f - sg, tt);
+              d3[t] = dav * silu;
+            }
+            pa[half * 8 + i / 2] = pack_bf16x2(av[0], av[1]);
+            pz1[half * 8 + i / 2] = pack_bf16x2(d1[0], d1[1]);
+            pz3[half * 8 + i / 2] = pack_bf16x2(d3[0], d3[1]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[BB_SL_EMPTY + slot]);
+        if (!waited_buf) {
+          if (!(ok = mbar_wait(&bars[BB_DZ_EMPTY], (j & 1) ^ 1, ab))) break;
+          waited_buf = true;
+        }
+        // hidden unit (within the slice) sc*32 + 8v + e  ->  atom sc/2, 16-byte chunk (sc%2)*4 + v
+        const uint32_t base = (sc >> 1) * 16384u;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t off = base + swz(row * 128 + ((sc & 1) * 4 + v) * 16, 128);
+          st_shared_v4(sa + off, pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
+          st_shared_v4(sdz1 + off, pz1[4 * v], pz1[4 * v + 1], pz1[4 * v + 2], pz1[4 * v + 3]);
+          st_shared_v4(sdz3 + off, pz3[4 * v], pz3[4 * v + 1], pz3[4 * v + 2], pz3[4 * v + 3]);
+        }
+      }
+      if (!ok) break;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BB_DZ_FULL]);
+    }
+    if (ok && cur_pair >= 0) dump(cur_pair);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace ttt

@@ -1,0 +1,360 @@
+// fwd.cuh — SwiGLU forward over token tiles on the 5th-gen tensor cores.
+//
+// Y = T_theta(X) = (silu(X W1) * (X W3)) W2 per head, for all n tokens
+// (VGG-T$^3$: Offline Feed-Forward 3D Reconstruction at Scale, Sec. 3.4,
+// Eq. 4 and "TTT MLP Architecture and Inner Optimization").
+//   READ mode : X = Q, writes O = Y (bf16).
+//   WRITE mode: X = K, writes the residual E = Y - V' (bf16); the backward
+//               kernel turns it into the gradient, the factor 2/n of the
+//               mean-squared loss is applied in the update.
+//
+// One persistent CTA per SM walks a contiguous range of (head, 128-token
+// tile) items.  Warp roles:
+//   warp 0   : TMA producer (weights of the current head by bulk copy, X and
+//              V' tiles by 2-D TMA, two stages each)
+//   warp 1   : TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2-9: two epilogue warpgroups
+// Per tile the hidden dimension is walked in chunks of 64 units:
+//   Z = X * [W1 | W3]_chunk      (M=128 tokens, N=128, K=d)   -> TMEM slot c%2
+//   A_chunk = silu(Z1) * Z3      (epilogue WG c%2, bf16, smem)
+//   Y += A_chunk * W2_chunk      (M=128, N=d, K=64)            -> TMEM Y slot
+// The MMA warp issues Z of chunk c+1 before Y of chunk c, so the tensor
+// pipe works while an epilogue warpgroup evaluates the gate.  The Y
+// epilogue of tile j runs (in warpgroup j%2) after that warpgroup's chunks
+// of tile j+1.
+#pragma once
+#include "sm100.cuh"
+
+namespace ttt {
+
+constexpr int kTileM = 128;
+constexpr int kThreads = 320;
+
+struct FwdParams {
+  const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
+  const __nv_bfloat16* w2_img;   // per head: HIDP rows of D bf16 (sw-swizzled)
+  __nv_bfloat16* out;            // [n][heads][D]
+  int n, heads, tiles;
+  unsigned int* status;
+};
+
+template <int D, int HIDP>
+struct FwdLayout {
+  static constexpr int SW = 2 * D;
+  static constexpr uint32_t kW13 = 2u * HIDP * D * 2;
+  static constexpr uint32_t kW2 = 1u * HIDP * D * 2;
+  static constexpr uint32_t kTile = 1u * kTileM * D * 2;
+  static constexpr uint32_t kA = kTileM * 64 * 2;
+  static constexpr uint32_t off_w13 = 0;
+  static constexpr uint32_t off_w2 = off_w13 + kW13;
+  static constexpr uint32_t off_x = off_w2 + kW2;
+  static constexpr uint32_t off_vp = off_x + 2 * kTile;
+  static constexpr uint32_t off_a = off_vp + 2 * kTile;
+  static constexpr uint32_t off_bar = off_a + 2 * kA;
+  static constexpr int kNumBars = 24;
+  static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
+  static_assert(off_x % 1024 == 0 && off_vp % 1024 == 0 && off_a % 1024 == 0, "1 KiB alignment");
+};
+
+// barrier indices
+enum FwdBar {
+  FB_W_FULL = 0, FB_W_EMPTY = 1, FB_X_FULL = 2, FB_X_EMPTY = 4, FB_VP_FULL = 6, FB_VP_EMPTY = 8,
+  FB_Z_FULL = 10, FB_Z_EMPTY = 12, FB_A_FULL = 14, FB_A_EMPTY = 16, FB_Y_FULL = 18, FB_Y_EMPTY = 20,
+  FB_DONE = 22
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Copy `bytes` (multiple of 16) from global to shared in 16 KiB bulk pieces.
+__device__ __forceinline__ void bulk_load_pieces(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  for (uint32_t o = 0; o < bytes; o += 16384u) {
+    const uint32_t len = bytes - o < 16384u ? bytes - o : 16384u;
+    bulk_load(static_cast<uint8_t*>(dst) + o, static_cast<const uint8_t*>(src) + o, len, bar);
+  }
+}
+
+// Bounded wait that ignores the abort flag (used only while draining).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitClockLimit) break;
+  }
+}
+
+template <int D, int HIDP, bool WRITE>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_vp,
+               const FwdParams p) {
+  using L = FwdLayout<D, HIDP>;
+  constexpr int SW = L::SW;
+  constexpr int NC = HIDP / 64;
+  static_assert(NC % 2 == 0, "hidden chunks are split between two warpgroups");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const Abort ab{abort_flag, p.status};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const long long total = static_cast<long long>(p.heads) * p.tiles;
+  const long long it0 = total * blockIdx.x / gridDim.x;
+  const long long it1 = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[FB_W_FULL], 1);
+    mbar_init(&bars[FB_W_EMPTY], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[FB_X_FULL + s], 1);
+      mbar_init(&bars[FB_X_EMPTY + s], 1);
+      mbar_init(&bars[FB_VP_FULL + s], 1);
+      mbar_init(&bars[FB_VP_EMPTY + s], 4);
+      mbar_init(&bars[FB_Z_FULL + s], 1);
+      mbar_init(&bars[FB_Z_EMPTY + s], 4);
+      mbar_init(&bars[FB_A_FULL + s], 4);
+      mbar_init(&bars[FB_A_EMPTY + s], 1);
+      mbar_init(&bars[FB_Y_FULL + s], 1);
+      mbar_init(&bars[FB_Y_EMPTY + s], 4);
+    }
+    mbar_init(&bars[FB_DONE], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tz = tbase;          // 2 Z slots x 128 columns
+  const uint32_t ty = tbase + 256;    // 2 Y slots x D columns
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_x);
+      if (WRITE) tma_prefetch_desc(&tm_vp);
+      int cur_head = -1;
+      uint32_t wl = 0, j = 0;
+      for (long long it = it0; it < it1; ++it, ++j) {
+        const int head = static_cast<int>(it / p.tiles);
+        const int tile = static_cast<int>(it % p.tiles);
+        if (head != cur_head) {
+          if (wl > 0 && !mbar_wait(&bars[FB_W_EMPTY], (wl - 1) & 1, ab)) break;
+          mbar_arrive_expect_tx(&bars[FB_W_FULL], L::kW13 + L::kW2);
+          bulk_load_pieces(smem + L::off_w13, p.w13_img + static_cast<size_t>(head) * (L::kW13 / 2), L::kW13,
+                           &bars[FB_W_FULL]);
+          bulk_load_pieces(smem + L::off_w2, p.w2_img + static_cast<size_t>(head) * (L::kW2 / 2), L::kW2,
+                           &bars[FB_W_FULL]);
+          ++wl;
+          cur_head = head;
+        }
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&bars[FB_X_EMPTY + s], ph ^ 1, ab)) break;
+        mbar_arrive_expect_tx(&bars[FB_X_FULL + s], L::kTile);
+        tma_load_2d(smem + L::off_x + s * L::kTile, &tm_x, &bars[FB_X_FULL + s], head * D, tile * kTileM);
+        if (WRITE) {
+          if (!mbar_wait(&bars[FB_VP_EMPTY + s], ph ^ 1, ab)) break;
+          mbar_arrive_expect_tx(&bars[FB_VP_FULL + s], L::kTile);
+          tma_load_2d(smem + L::off_vp + s * L::kTile, &tm_vp, &bars[FB_VP_FULL + s], head * D, tile * kTileM);
+        }
+      }
+      // Drain: the last load issued into each barrier has landed before exit.
+      if (wl > 0) mbar_drain(&bars[FB_W_FULL], (wl - 1) & 1);
+      for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) {
+        mbar_drain(&bars[FB_X_FULL + (jj & 1)], (jj >> 1) & 1);
+        if (WRITE) mbar_drain(&bars[FB_VP_FULL + (jj & 1)], (jj >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdZ = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdY = idesc_bf16(128, D, false, true);
+      const uint32_t w13 = smem_u32(smem + L::off_w13);
+      const uint32_t w2 = smem_u32(smem + L::off_w2);
+      int cur_head = -1;
+      uint32_t wl = 0, j = 0, zc = 0;
+      bool pend = false, ok = true;
+      uint32_t pend_j = 0;
+      int pend_c = 0;
+      // Y += A_chunk * W2_chunk for a chunk whose gate the epilogue has written.
+      auto issue_y = [&](uint32_t qj, int qc) -> bool {
+        const uint32_t ys = qj & 1;
+        if (qc == 0 && !mbar_wait(&bars[FB_Y_EMPTY + ys], ((qj >> 1) & 1) ^ 1, ab)) return false;
+        const int g = qc & 1;
+        const uint32_t u = qj * (NC / 2) + (qc >> 1);
+        if (!mbar_wait(&bars[FB_A_FULL + g], u & 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = smem_desc(abuf + 32 * k, 0, 1024, 128);
+          const uint64_t bd = smem_desc(w2 + (64 * qc + 16 * k) * SW, HIDP * SW, 8 * SW, SW);
+          mma_bf16(ty + ys * D, ad, bd, kIdY, (qc > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars[FB_A_EMPTY + g]);
+        if (qc == NC - 1) mma_commit(&bars[FB_Y_FULL + ys]);
+        return true;
+      };
+      for (long long it = it0; it < it1 && ok; ++it, ++j) {
+        const int head = static_cast<int>(it / p.tiles);
+        if (head != cur_head) {
+          if (pend) {
+            if (!(ok = issue_y(pend_j, pend_c))) break;
+            pend = false;
+          }
+          if (cur_head >= 0) mma_commit(&bars[FB_W_EMPTY]);
+          if (!(ok = mbar_wait(&bars[FB_W_FULL], wl & 1, ab))) break;
+          ++wl;
+          cur_head = head;
+        }
+        const int s = j & 1;
+        if (!(ok = mbar_wait(&bars[FB_X_FULL + s], (j >> 1) & 1, ab))) break;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + L::off_x + s * L::kTile);
+        for (int c = 0; c < NC; ++c) {
+          const int zs = c & 1;
+          const uint32_t use = zc >> 1;
+          if (!(ok = mbar_wait(&bars[FB_Z_EMPTY + zs], (use & 1) ^ 1, ab))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t ad = smem_desc(xa + 32 * k, 0, 8 * SW, SW);
+            const uint64_t bd = smem_desc(w13 + 128 * c * SW + 32 * k, 0, 8 * SW, SW);
+            mma_bf16(tz + zs * 128, ad, bd, kIdZ, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars[FB_Z_FULL + zs]);
+          if (c == NC - 1) mma_commit(&bars[FB_X_EMPTY + s]);
+          ++zc;
+          if (pend && !(ok = issue_y(pend_j, pend_c))) break;
+          pend = true;
+          pend_j = j;
+          pend_c = c;
+        }
+      }
+      if (ok && pend) issue_y(pend_j, pend_c);
+      // All issued MMAs have completed before TMEM is released.
+      mma_commit(&bars[FB_DONE]);
+      mbar_drain(&bars[FB_DONE], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int g = (warp - 2) >> 2;          // warpgroup
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;          // token row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
+    uint32_t j = 0, u = 0;
+    long long prev_it = -1;
+
+    // Y epilogue of tile jj (item `itj`), done by warpgroup jj % 2.
+    auto y_epilogue = [&](uint32_t jj, long long itj) -> bool {
+      const int head = static_cast<int>(itj / p.tiles);
+      const int tile = static_cast<int>(itj % p.tiles);
+      const uint32_t ys = jj & 1;
+      if (!mbar_wait(&bars[FB_Y_FULL + ys], (jj >> 1) & 1, ab)) return false;
+      tc_fence_after();
+      float y[D];
+      const uint32_t yb = ty + ys * D + lane_off;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        if (D >= 16 && c0 + 16 <= D) {
+          uint32_t r[16];
+          tmem_ld16(yb + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[c0 + i] = __uint_as_float(r[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[FB_Y_EMPTY + ys]);
+      if (WRITE) {
+        if (!mbar_wait(&bars[FB_VP_FULL + ys], (jj >> 1) & 1, ab)) return false;
+        const uint32_t vb = smem_u32(smem + L::off_vp + ys * L::kTile);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) {
+          uint32_t v0, v1, v2, v3;
+          ld_shared_v4(vb + swz(row * SW + ch * 16, SW), v0, v1, v2, v3);
+          y[8 * ch + 0] -= bf16lo(v0); y[8 * ch + 1] -= bf16hi(v0);
+          y[8 * ch + 2] -= bf16lo(v1); y[8 * ch + 3] -= bf16hi(v1);
+          y[8 * ch + 4] -= bf16lo(v2); y[8 * ch + 5] -= bf16hi(v2);
+          y[8 * ch + 6] -= bf16lo(v3); y[8 * ch + 7] -= bf16hi(v3);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[FB_VP_EMPTY + ys]);
+      }
+      const long long tok = static_cast<long long>(tile) * kTileM + row;
+      if (tok < p.n) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + head) * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) {
+          uint4 v;
+          v.x = pack_bf16x2(y[8 * ch + 0], y[8 * ch + 1]);
+          v.y = pack_bf16x2(y[8 * ch + 2], y[8 * ch + 3]);
+          v.z = pack_bf16x2(y[8 * ch + 4], y[8 * ch + 5]);
+          v.w = pack_bf16x2(y[8 * ch + 6], y[8 * ch + 7]);
+          dst[ch] = v;
+        }
+      }
+      return true;
+    };
+
+    bool ok = true;
+    for (long long it = it0; it < it1 && ok; ++it, ++j) {
+      for (int c = g; c < NC; c += 2, ++u) {
+        if (!(ok = mbar_wait(&bars[FB_Z_FULL + g], u & 1, ab))) break;
+        tc_fence_after();
+        uint32_t apk[32];  // 64 gate values of this row, bf16 pairs
+        const uint32_t zb = tz + g * 128 + lane_off;
+#pragma unroll
+        for (int sc = 0; sc < 2; ++sc) {
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            uint32_t z1[16], z3[16];
+            tmem_ld16(zb + sc * 64 + qq * 16, z1);
+            tmem_ld16(zb + sc * 64 + 32 + qq * 16, z3);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const float a0 = __uint_as_float(z1[i]), a1 = __uint_as_float(z1[i + 1]);
+              const float b0 = __uint_as_float(z3[i]), b1 = __uint_as_float(z3[i + 1]);
+              apk[(sc * 2 + qq) * 8 + i / 2] =
+                  pack_bf16x2(a0 * sigmoid_fast(a0) * b0, a1 * sigmoid_fast(a1) * b1);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + g]);
+        if (!(ok = mbar_wait(&bars[FB_A_EMPTY + g], (u & 1) ^ 1, ab))) break;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(abuf + swz(row * 128 + ch * 16, 128), apk[4 * ch], apk[4 * ch + 1], apk[4 * ch + 2],
+                       apk[4 * ch + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[FB_A_FULL + g]);
+      }
+      if (!ok) break;
+      if (j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) ok = y_epilogue(j - 1, prev_it);
+      prev_it = it;
+    }
+    if (ok && j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) y_epilogue(j - 1, prev_it);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace ttt

@@ -1,0 +1,538 @@
+// ttt_capi.cu — the C ABI declared in include/ttt.h: host-side validation,
+// workspace layout, TMA descriptors and the launch sequence of the layer
+//   conv -> steps x [pack theta -> forward (residual) -> backward (partials)
+//   -> reduce + SGD] -> pack theta* -> forward (read).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/ttt.h"
+#include "conv.cuh"
+#include "update.cuh"
+
+using namespace ttt;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+struct Shape {
+  long long n;   // tokens
+  int H, D, h, hidp, tiles, slices;
+  long long C;   // H * D channels
+};
+
+int check_dims(const ttt_dims* dm, Shape* s) {
+  if (!dm) return TTT_EINVAL;
+  if (dm->n_views < 1 || dm->grid_h < 1 || dm->grid_w < 1 || dm->n_special < 0 || dm->heads < 1 || dm->d < 1 ||
+      dm->h < 1)
+    return TTT_EINVAL;
+  if (!(dm->d == 16 || dm->d == 32 || dm->d == 64)) return TTT_EUNSUPPORTED;
+  if (dm->h > 256) return TTT_EUNSUPPORTED;
+  const long long T = static_cast<long long>(dm->n_special) + static_cast<long long>(dm->grid_h) * dm->grid_w;
+  const long long n = T * dm->n_views;
+  if (n <= 0 || n > (1LL << 31) - 1 - 128) return TTT_EUNSUPPORTED;   // TMA coordinates are int32
+  if (dm->n_views > 65535 || dm->grid_h > 65534) return TTT_EUNSUPPORTED;  // conv grid limits
+  s->n = n;
+  s->H = dm->heads;
+  s->D = dm->d;
+  s->h = dm->h;
+  s->hidp = (dm->h + 127) / 128 * 128;
+  s->slices = s->hidp / 128;
+  s->tiles = static_cast<int>((n + kTileM - 1) / kTileM);
+  s->C = static_cast<long long>(dm->heads) * dm->d;
+  return TTT_OK;
+}
+
+int num_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+struct Grids {
+  int fwd, bwd, max_contrib;
+};
+
+Grids grids_for(const Shape& s, int sms) {
+  Grids g;
+  const long long fi = static_cast<long long>(s.H) * s.tiles;
+  const long long bi = static_cast<long long>(s.H) * s.slices * s.tiles;
+  g.fwd = static_cast<int>(std::min<long long>(sms, fi));
+  g.bwd = static_cast<int>(std::min<long long>(sms, bi));
+  int mc = 1;
+  for (long long pair = 0; pair < static_cast<long long>(s.H) * s.slices; ++pair) {
+    const long long lo = owner_cta(pair * s.tiles, bi, g.bwd);
+    const long long hi = owner_cta(pair * s.tiles + s.tiles - 1, bi, g.bwd);
+    mc = std::max<int>(mc, static_cast<int>(hi - lo + 1));
+  }
+  g.max_contrib = mc;
+  return g;
+}
+
+struct Ws {
+  size_t status, w13, w2, vp, e, part, q, k, v, o, convw, th0, thout, total;
+};
+
+Ws ws_layout(const Shape& s, const Grids& g, int op) {
+  Ws w;
+  memset(&w, 0, sizeof(w));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = off;
+    off = align_up(off + bytes);
+    return r;
+  };
+  const size_t tok_bytes = static_cast<size_t>(s.n) * s.C * 2;
+  const size_t theta_bytes = 3ull * s.H * s.D * s.h * 4;
+  w.status = take(256);
+  w.w13 = take(static_cast<size_t>(s.H) * 2 * s.hidp * s.D * 2);
+  w.w2 = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
+  if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST) {
+    w.vp = take(tok_bytes);
+    w.e = take(tok_bytes);
+    w.part = take(static_cast<size_t>(s.H) * s.slices * g.max_contrib * 3ull * 128 * s.D * 4);
+  }
+  if (op == TTT_OP_LAYER_HOST) {
+    w.q = take(tok_bytes);
+    w.k = take(tok_bytes);
+    w.v = take(tok_bytes);
+    w.o = take(tok_bytes);
+    w.convw = take(static_cast<size_t>(s.C) * 9 * 4);
+    w.th0 = take(theta_bytes);
+    w.thout = take(theta_bytes);
+  }
+  w.total = off;
+  return w;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D view [n rows][C bf16] of a token tensor; box = D columns x 128 rows,
+// swizzled by rows of 2*D bytes (the layout the kernels' descriptors expect).
+bool make_token_map(CUtensorMap* m, const void* base, const Shape& s) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(s.C), static_cast<cuuint64_t>(s.n)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(s.C) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(s.D), static_cast<cuuint32_t>(kTileM)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = s.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                          : (s.D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ profiling
+enum KernelKind { KK_CONV = 0, KK_PACK = 1, KK_FWD_WRITE = 2, KK_BWD = 3, KK_REDUCE = 4, KK_FWD_READ = 5 };
+const char* const kKernelNames[TTT_KERNEL_KINDS] = {"shortconv2d", "pack_theta", "swiglu_fwd_residual",
+                                                     "swiglu_bwd_partials", "reduce_sgd", "swiglu_fwd_read"};
+constexpr size_t kMaxProfiled = 65536;
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> ev;   // 2 per launch
+  std::vector<int> kind;
+  size_t used = 0;
+  int dropped = 0;
+};
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+
+// Records an event pair around one launch when profiling is on.
+struct ProfScope {
+  cudaEvent_t end = nullptr;
+  cudaStream_t st;
+  ProfScope(int k, cudaStream_t s) : st(s) {
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (!p.on) return;
+    if (p.used >= kMaxProfiled) {
+      ++p.dropped;
+      return;
+    }
+    while (p.ev.size() < 2 * (p.used + 1)) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      p.ev.push_back(e);
+    }
+    if (p.kind.size() < p.used + 1) p.kind.resize(p.used + 1);
+    p.kind[p.used] = k;
+    cudaEventRecord(p.ev[2 * p.used], st);
+    end = p.ev[2 * p.used + 1];
+    ++p.used;
+  }
+  ~ProfScope() {
+    if (end) cudaEventRecord(end, st);
+  }
+};
+
+bool aligned(const void* p, size_t a = 16) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ECUDA; }
+
+// ------------------------------------------------------------------ launches
+int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float* w, uint16_t* out,
+             cudaStream_t st) {
+  ConvParams p;
+  p.V = reinterpret_cast<const uint4*>(V);
+  p.w = w;
+  p.out = reinterpret_cast<uint4*>(out);
+  p.n_views = dm->n_views;
+  p.gh = dm->grid_h;
+  p.gw = dm->grid_w;
+  p.n_special = dm->n_special;
+  p.C = static_cast<int>(s.C);
+  const int g8 = p.C / 8;
+  const int block = std::min(128, (g8 + 31) / 32 * 32);
+  dim3 grid((g8 + block - 1) / block, dm->grid_h + 1, dm->n_views);
+  ProfScope prof(KK_CONV, st);
+  shortconv_kernel<<<grid, block, 0, st>>>(p);
+  return launch_status();
+}
+
+int run_pack(const Shape& s, const float* theta, const Ws& w, uint8_t* ws, cudaStream_t st) {
+  PackParams p;
+  p.theta = theta;
+  p.w13_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w13);
+  p.w2_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w2);
+  p.heads = s.H;
+  p.d = s.D;
+  p.h = s.h;
+  p.hidp = s.hidp;
+  const long long total = static_cast<long long>(s.H) * 3 * s.hidp * s.D;
+  ProfScope prof(KK_PACK, st);
+  pack_images_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(p);
+  return launch_status();
+}
+
+// The tensor-core kernels allocate all 512 TMEM columns of their SM; asking
+// for more than half of the SM's shared memory keeps their residency at one
+// CTA per SM, so an allocation never waits for a co-resident CTA.
+constexpr uint32_t kHalfSmem = 116u * 1024u;
+uint32_t one_cta_per_sm(uint32_t bytes) { return bytes > kHalfSmem ? bytes : kHalfSmem; }
+
+template <int D, int HIDP, bool WRITE>
+int launch_fwd_t(const CUtensorMap& tx, const CUtensorMap& tvp, const FwdParams& p, int grid, cudaStream_t st) {
+  using L = FwdLayout<D, HIDP>;
+  auto k = fwd_kernel<D, HIDP, WRITE>;
+  const uint32_t smem = one_cta_per_sm(L::bytes);
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTT_ECUDA;
+  ProfScope prof(WRITE ? KK_FWD_WRITE : KK_FWD_READ, st);
+  k<<<grid, kThreads, smem, st>>>(tx, tvp, p);
+  return launch_status();
+}
+
+template <bool WRITE>
+int launch_fwd(const Shape& s, const CUtensorMap& tx, const CUtensorMap& tvp, const FwdParams& p, int grid,
+               cudaStream_t st) {
+#define TTT_FWD_CASE(DD, HH) \
+  if (s.D == DD && s.hidp == HH) return launch_fwd_t<DD, HH, WRITE>(tx, tvp, p, grid, st);
+  TTT_FWD_CASE(16, 128) TTT_FWD_CASE(16, 256) TTT_FWD_CASE(32, 128) TTT_FWD_CASE(32, 256)
+  TTT_FWD_CASE(64, 128) TTT_FWD_CASE(64, 256)
+#undef TTT_FWD_CASE
+  return TTT_EUNSUPPORTED;
+}
+
+template <int D>
+int launch_bwd_t(const CUtensorMap& tk, const CUtensorMap& te, const BwdParams& p, int grid, cudaStream_t st) {
+  using L = BwdLayout<D>;
+  auto k = bwd_kernel<D>;
+  const uint32_t smem = one_cta_per_sm(L::bytes);
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return TTT_ECUDA;
+  ProfScope prof(KK_BWD, st);
+  k<<<grid, kThreads, smem, st>>>(tk, te, p);
+  return launch_status();
+}
+
+int launch_bwd(const Shape& s, const CUtensorMap& tk, const CUtensorMap& te, const BwdParams& p, int grid,
+               cudaStream_t st) {
+  if (s.D == 16) return launch_bwd_t<16>(tk, te, p, grid, st);
+  if (s.D == 32) return launch_bwd_t<32>(tk, te, p, grid, st);
+  if (s.D == 64) return launch_bwd_t<64>(tk, te, p, grid, st);
+  return TTT_EUNSUPPORTED;
+}
+
+struct Call {
+  Shape s;
+  Grids g;
+  Ws w;
+  uint8_t* ws;
+  cudaStream_t st;
+};
+
+// Host-side validation first (no CUDA call), then the device-dependent sizes.
+int prepare(const ttt_dims* dm, int op, void* workspace, size_t ws_bytes, void* stream, Call* c) {
+  int rc = check_dims(dm, &c->s);
+  if (rc != TTT_OK) return rc;
+  if (!workspace) return TTT_EINVAL;
+  if (!aligned(workspace, 256)) return TTT_EALIGN;
+  const int sms = num_sms();
+  if (sms <= 0) return TTT_ECUDA;
+  c->g = grids_for(c->s, sms);
+  c->w = ws_layout(c->s, c->g, op);
+  if (ws_bytes < c->w.total) return TTT_EWORKSPACE;
+  c->ws = static_cast<uint8_t*>(workspace);
+  c->st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(c->ws + c->w.status, 0, 4, c->st) != cudaSuccess) return TTT_ECUDA;
+  return TTT_OK;
+}
+
+int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
+              const float* theta0, float lr, int steps, float* theta_out) {
+  const Shape& s = c.s;
+  uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
+  uint16_t* e = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
+  unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
+  if (rc != TTT_OK) return rc;
+  if (steps == 0) {
+    if (theta_out != theta0 &&
+        cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    return TTT_OK;
+  }
+  CUtensorMap tk, tvp, te;
+  if (!make_token_map(&tk, K, s) || !make_token_map(&tvp, vp, s) || !make_token_map(&te, e, s)) return TTT_ECUDA;
+  FwdParams fp;
+  fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
+  fp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
+  fp.out = reinterpret_cast<__nv_bfloat16*>(e);
+  fp.n = static_cast<int>(s.n);
+  fp.heads = s.H;
+  fp.tiles = s.tiles;
+  fp.status = status;
+  BwdParams bp;
+  bp.w13_img = fp.w13_img;
+  bp.w2_img = fp.w2_img;
+  bp.partials = reinterpret_cast<float*>(c.ws + c.w.part);
+  bp.n = fp.n;
+  bp.heads = s.H;
+  bp.tiles = s.tiles;
+  bp.slices = s.slices;
+  bp.max_contrib = c.g.max_contrib;
+  bp.status = status;
+  UpdateParams up;
+  up.partials = bp.partials;
+  up.theta_out = theta_out;
+  up.heads = s.H;
+  up.d = s.D;
+  up.h = s.h;
+  up.slices = s.slices;
+  up.tiles = s.tiles;
+  up.max_contrib = c.g.max_contrib;
+  up.n_items = static_cast<long long>(s.H) * s.slices * s.tiles;
+  up.grid = c.g.bwd;
+  up.scale = lr * 2.0f / static_cast<float>(s.n);
+  const long long red_threads = static_cast<long long>(s.H) * s.slices * 3 * 128 * s.D;
+  for (int step = 0; step < steps; ++step) {
+    const float* th_in = step == 0 ? theta0 : theta_out;
+    if ((rc = run_pack(s, th_in, c.w, c.ws, c.st)) != TTT_OK) return rc;
+    if ((rc = launch_fwd<true>(s, tk, tvp, fp, c.g.fwd, c.st)) != TTT_OK) return rc;
+    if ((rc = launch_bwd(s, tk, te, bp, c.g.bwd, c.st)) != TTT_OK) return rc;
+    up.theta_in = th_in;
+    {
+      ProfScope prof(KK_REDUCE, c.st);
+      reduce_sgd_kernel<<<static_cast<unsigned>((red_threads + 255) / 256), 256, 0, c.st>>>(up);
+    }
+    if ((rc = launch_status()) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
+int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
+  const Shape& s = c.s;
+  int rc = run_pack(s, theta, c.w, c.ws, c.st);
+  if (rc != TTT_OK) return rc;
+  CUtensorMap tq;
+  if (!make_token_map(&tq, Q, s)) return TTT_ECUDA;
+  FwdParams fp;
+  fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
+  fp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
+  fp.out = reinterpret_cast<__nv_bfloat16*>(O);
+  fp.n = static_cast<int>(s.n);
+  fp.heads = s.H;
+  fp.tiles = s.tiles;
+  fp.status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
+  return launch_fwd<false>(s, tq, tq, fp, c.g.fwd, c.st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttt_workspace_bytes(const ttt_dims* dims, int op) {
+  Shape s;
+  if (check_dims(dims, &s) != TTT_OK) return 0;
+  if (op < TTT_OP_WRITE || op > TTT_OP_LAYER_HOST) return 0;
+  const int sms = num_sms();
+  if (sms <= 0) return 0;
+  return ws_layout(s, grids_for(s, sms), op).total;
+}
+
+int ttt_shortconv2d(const ttt_dims* dims, const uint16_t* V, const float* conv_w, uint16_t* V_out, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != TTT_OK) return rc;
+  if (!V || !conv_w || !V_out) return TTT_EINVAL;
+  if (!aligned(V) || !aligned(conv_w) || !aligned(V_out)) return TTT_EALIGN;
+  return run_conv(s, dims, V, conv_w, V_out, static_cast<cudaStream_t>(stream));
+}
+
+int ttt_write(const ttt_dims* dims, const uint16_t* K, const uint16_t* V, const float* conv_w, const float* theta0,
+              float lr, int steps, float* theta_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!K || !V || !conv_w || !theta0 || !theta_out || steps < 0) return TTT_EINVAL;
+  if (!aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out)) return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  return run_write(c, dims, K, V, conv_w, theta0, lr, steps, theta_out);
+}
+
+int ttt_read(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O, void* workspace,
+             size_t workspace_bytes, void* stream) {
+  if (!Q || !theta || !O) return TTT_EINVAL;
+  if (!aligned(Q) || !aligned(theta) || !aligned(O)) return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_READ, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  return run_read(c, Q, theta, O);
+}
+
+int ttt_layer(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const uint16_t* V, const float* conv_w,
+              const float* theta0, float lr, int steps, float* theta_out, uint16_t* O, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !conv_w || !theta0 || !theta_out || !O || steps < 0) return TTT_EINVAL;
+  if (!aligned(Q) || !aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out) ||
+      !aligned(O))
+    return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  if ((rc = run_write(c, dims, K, V, conv_w, theta0, lr, steps, theta_out)) != TTT_OK) return rc;
+  return run_read(c, Q, theta_out, O);
+}
+
+int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t* K_host, const uint16_t* V_host,
+                   const float* conv_w_host, const float* theta0_host, float lr, int steps, float* theta_out_host,
+                   uint16_t* O_host, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q_host || !K_host || !V_host || !conv_w_host || !theta0_host || !theta_out_host || !O_host || steps < 0)
+    return TTT_EINVAL;
+  Call c;
+  int rc = prepare(dims, TTT_OP_LAYER_HOST, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  const Shape& s = c.s;
+  const size_t tok = static_cast<size_t>(s.n) * s.C * 2;
+  const size_t thb = 3ull * s.H * s.D * s.h * 4;
+  uint16_t* dq = reinterpret_cast<uint16_t*>(c.ws + c.w.q);
+  uint16_t* dk = reinterpret_cast<uint16_t*>(c.ws + c.w.k);
+  uint16_t* dv = reinterpret_cast<uint16_t*>(c.ws + c.w.v);
+  uint16_t* dout = reinterpret_cast<uint16_t*>(c.ws + c.w.o);
+  float* dw = reinterpret_cast<float*>(c.ws + c.w.convw);
+  float* dth0 = reinterpret_cast<float*>(c.ws + c.w.th0);
+  float* dthout = reinterpret_cast<float*>(c.ws + c.w.thout);
+  if (cudaMemcpyAsync(dq, Q_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+      cudaMemcpyAsync(dk, K_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+      cudaMemcpyAsync(dv, V_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+      cudaMemcpyAsync(dw, conv_w_host, static_cast<size_t>(s.C) * 9 * 4, cudaMemcpyHostToDevice, c.st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(dth0, theta0_host, thb, cudaMemcpyHostToDevice, c.st) != cudaSuccess)
+    return TTT_ECUDA;
+  if ((rc = run_write(c, dims, dk, dv, dw, dth0, lr, steps, dthout)) != TTT_OK) return rc;
+  if ((rc = run_read(c, dq, dthout, dout)) != TTT_OK) return rc;
+  if (cudaMemcpyAsync(theta_out_host, dthout, thb, cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
+      cudaMemcpyAsync(O_host, dout, tok, cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
+    return TTT_ECUDA;
+  return TTT_OK;
+}
+
+int ttt_check_status(const void* workspace, void* stream) {
+  if (!workspace) return TTT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ECUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ECUDA;
+  if (v != 0) {
+    if (cudaMemset(const_cast<void*>(workspace), 0, 4) != cudaSuccess) return TTT_ECUDA;
+    return TTT_EDEVICE;
+  }
+  return TTT_OK;
+}
+
+int ttt_profile_start(void) {
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  p.on = true;
+  p.used = 0;
+  p.dropped = 0;
+  return TTT_OK;
+}
+
+int ttt_profile_stop(ttt_kernel_times* out) {
+  if (!out) return TTT_EINVAL;
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  p.on = false;
+  memset(out, 0, sizeof(*out));
+  int rc = TTT_OK;
+  for (size_t i = 0; i < p.used; ++i) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(p.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]) != cudaSuccess) {
+      rc = TTT_ECUDA;
+      continue;
+    }
+    out->launches[p.kind[i]] += 1;
+    out->total_ms[p.kind[i]] += ms;
+  }
+  out->dropped = p.dropped;
+  p.used = 0;
+  return rc;
+}
+
+const char* ttt_kernel_name(int kind) {
+  return (kind >= 0 && kind < TTT_KERNEL_KINDS) ? kKernelNames[kind] : "unknown";
+}
+
+const char* ttt_status_str(int status) {
+  switch (status) {
+    case TTT_OK: return "ok";
+    case TTT_EINVAL: return "invalid argument";
+    case TTT_EALIGN: return "misaligned pointer";
+    case TTT_EUNSUPPORTED: return "unsupported shape";
+    case TTT_EWORKSPACE: return "workspace too small";
+    case TTT_ECUDA: return "CUDA error";
+    case TTT_EDEVICE: return "device-side fault recorded";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

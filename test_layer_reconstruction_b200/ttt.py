@@ -1,0 +1,220 @@
+"""Python binding of the C ABI in include/ttt.h (argument marshalling only).
+
+Every step of the layer runs in the CUDA kernels of libttt.so; PyTorch only
+provides device memory and the current stream.  There is no fallback: if the
+library is not built, or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple, Union
+
+import torch
+
+from .inputs import LayerConfig
+
+__all__ = [
+    "TTTError", "Dims", "library_path", "load_library", "workspace_bytes", "make_workspace",
+    "shortconv2d", "write", "read", "layer", "layer_host", "check_status",
+    "OP_WRITE", "OP_READ", "OP_LAYER", "OP_LAYER_HOST", "EXPORTED_SYMBOLS", "profile_start", "profile_stop",
+]
+
+OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
+EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
+                    "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
+                    "ttt_profile_stop", "ttt_kernel_name")
+KERNEL_KINDS = 6
+
+
+class KernelTimes(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int32 * KERNEL_KINDS), ("total_ms", ctypes.c_float * KERNEL_KINDS),
+                ("dropped", ctypes.c_int32)]
+
+
+class Dims(ctypes.Structure):
+    """ttt_dims: token layout and fast-weight shape."""
+    _fields_ = [("n_views", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("n_special", ctypes.c_int32), ("heads", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("h", ctypes.c_int32)]
+
+    @classmethod
+    def of(cls, x: Union["Dims", LayerConfig, dict]) -> "Dims":
+        if isinstance(x, Dims):
+            return x
+        if isinstance(x, LayerConfig):
+            x = x.dims()
+        return cls(**{k: int(x[k]) for k in ("n_views", "grid_h", "grid_w", "n_special", "heads", "d", "h")})
+
+    @property
+    def n(self) -> int:
+        return self.n_views * (self.n_special + self.grid_h * self.grid_w)
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttt.so")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libttt.so (built by ``python -m test_layer_reconstruction_b200.build``)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -m test_layer_reconstruction_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, S, F, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+    DP = ctypes.POINTER(Dims)
+    lib.ttt_workspace_bytes.argtypes = [DP, I]
+    lib.ttt_workspace_bytes.restype = S
+    lib.ttt_shortconv2d.argtypes = [DP, P, P, P, P]
+    lib.ttt_write.argtypes = [DP, P, P, P, P, F, I, P, P, S, P]
+    lib.ttt_read.argtypes = [DP, P, P, P, P, S, P]
+    lib.ttt_layer.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
+    lib.ttt_layer_host.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
+    lib.ttt_check_status.argtypes = [P, P]
+    lib.ttt_status_str.argtypes = [I]
+    lib.ttt_status_str.restype = ctypes.c_char_p
+    lib.ttt_profile_start.argtypes = []
+    lib.ttt_profile_stop.argtypes = [ctypes.POINTER(KernelTimes)]
+    lib.ttt_kernel_name.argtypes = [I]
+    lib.ttt_kernel_name.restype = ctypes.c_char_p
+    for f in ("ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer", "ttt_layer_host", "ttt_check_status",
+              "ttt_profile_start", "ttt_profile_stop"):
+        getattr(lib, f).restype = I
+    _LIB = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    try:
+        return load_library().ttt_status_str(status).decode()
+    except Exception:  # pragma: no cover
+        return "unknown"
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise TTTError(rc, what)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def workspace_bytes(dims, op: int) -> int:
+    return int(load_library().ttt_workspace_bytes(ctypes.byref(Dims.of(dims)), op))
+
+
+def make_workspace(dims, op: int, device="cuda") -> torch.Tensor:
+    nb = workspace_bytes(dims, op)
+    if nb == 0:
+        raise TTTError(-3, "ttt_workspace_bytes")
+    return torch.empty(nb, dtype=torch.uint8, device=device)
+
+
+def shortconv2d(V: torch.Tensor, conv_w: torch.Tensor, dims, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """V' = ShortConv2D(V); V, out: bf16 [n, heads, d]; conv_w: f32 [heads*d, 3, 3]."""
+    dm = Dims.of(dims)
+    out = torch.empty_like(V) if out is None else out
+    _check(load_library().ttt_shortconv2d(ctypes.byref(dm), _dev(V, torch.bfloat16, "V"),
+                                          _dev(conv_w, torch.float32, "conv_w"),
+                                          _dev(out, torch.bfloat16, "out"), _stream()), "ttt_shortconv2d")
+    return out
+
+
+def write(K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, workspace=None) -> torch.Tensor:
+    """theta* after `steps` SGD steps on the TTT loss (Eq. 3); returns theta_out."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta0) if theta_out is None else theta_out
+    ws = make_workspace(dm, OP_WRITE, K.device) if workspace is None else workspace
+    _check(load_library().ttt_write(ctypes.byref(dm), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V"),
+                                    _dev(conv_w, torch.float32, "conv_w"), _dev(theta0, torch.float32, "theta0"),
+                                    float(lr), int(steps), _dev(theta_out, torch.float32, "theta_out"),
+                                    ws.data_ptr(), ws.numel(), _stream()), "ttt_write")
+    return theta_out
+
+
+def read(Q, theta, dims, O=None, workspace=None) -> torch.Tensor:
+    """O = T_theta(Q) (Eq. 4) with frozen theta."""
+    dm = Dims.of(dims)
+    O = torch.empty_like(Q) if O is None else O
+    ws = make_workspace(dm, OP_READ, Q.device) if workspace is None else workspace
+    _check(load_library().ttt_read(ctypes.byref(dm), _dev(Q, torch.bfloat16, "Q"),
+                                   _dev(theta, torch.float32, "theta"), _dev(O, torch.bfloat16, "O"),
+                                   ws.data_ptr(), ws.numel(), _stream()), "ttt_read")
+    return O
+
+
+def layer(Q, K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, O=None,
+          workspace=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The whole TTT layer; returns (theta*, O)."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta0) if theta_out is None else theta_out
+    O = torch.empty_like(Q) if O is None else O
+    ws = make_workspace(dm, OP_LAYER, Q.device) if workspace is None else workspace
+    _check(load_library().ttt_layer(ctypes.byref(dm), _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"),
+                                    _dev(V, torch.bfloat16, "V"), _dev(conv_w, torch.float32, "conv_w"),
+                                    _dev(theta0, torch.float32, "theta0"), float(lr), int(steps),
+                                    _dev(theta_out, torch.float32, "theta_out"), _dev(O, torch.bfloat16, "O"),
+                                    ws.data_ptr(), ws.numel(), _stream()), "ttt_layer")
+    return theta_out, O
+
+
+def _host(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor of {dtype}")
+    return t.data_ptr()
+
+
+def layer_host(Q, K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out, O, workspace) -> None:
+    """ttt_layer on host (preferably pinned) tensors; enqueued on the current stream."""
+    dm = Dims.of(dims)
+    _check(load_library().ttt_layer_host(ctypes.byref(dm), _host(Q, torch.bfloat16, "Q"),
+                                         _host(K, torch.bfloat16, "K"), _host(V, torch.bfloat16, "V"),
+                                         _host(conv_w, torch.float32, "conv_w"),
+                                         _host(theta0, torch.float32, "theta0"), float(lr), int(steps),
+                                         _host(theta_out, torch.float32, "theta_out"),
+                                         _host(O, torch.bfloat16, "O"), workspace.data_ptr(), workspace.numel(),
+                                         _stream()), "ttt_layer_host")
+
+
+def check_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream and return the workspace's device status (0 = ok)."""
+    return int(load_library().ttt_check_status(ctypes.c_void_p(workspace.data_ptr()), _stream()))
+
+
+def profile_start() -> None:
+    """Start recording a CUDA event pair around every kernel the library launches."""
+    _check(load_library().ttt_profile_start(), "ttt_profile_start")
+
+
+def profile_stop() -> dict:
+    """Stop recording; return {kernel name: {"launches": L, "total_ms": T}} (synchronises the events)."""
+    lib = load_library()
+    kt = KernelTimes()
+    _check(lib.ttt_profile_stop(ctypes.byref(kt)), "ttt_profile_stop")
+    out = {lib.ttt_kernel_name(k).decode(): {"launches": int(kt.launches[k]), "total_ms": float(kt.total_ms[k])}
+           for k in range(KERNEL_KINDS)}
+    out["_dropped"] = int(kt.dropped)
+    return out

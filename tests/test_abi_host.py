@@ -1,0 +1,71 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from test_layer_reconstruction_b200 import build, ttt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ttt.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "ttt.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_bound_symbols():
+    assert _declared_functions() == sorted(ttt.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(0, -7, -1):
+        assert ttt.status_str(code) != "unknown status"
+    assert ttt.status_str(-99) == "unknown status"
+
+
+def _dims(**kw):
+    base = dict(n_views=2, grid_h=8, grid_w=8, n_special=0, heads=1, d=16, h=32)
+    base.update(kw)
+    return ttt.Dims(**base)
+
+
+FAKE = ctypes.c_void_p(0x10000)       # never dereferenced: validation fails first
+FAKE_MIS = ctypes.c_void_p(0x10008)   # 8-byte aligned, not 16
+
+
+def _write(lib, dims, K=FAKE, ws=FAKE, steps=1):
+    return lib.ttt_write(ctypes.byref(dims), K, FAKE, FAKE, FAKE, 0.1, steps, FAKE, ws, 1 << 20, None)
+
+
+def test_host_validation_codes(lib):
+    assert _write(lib, _dims(), K=None) == -1                       # null pointer
+    assert _write(lib, _dims(), steps=-1) == -1                     # negative steps
+    assert _write(lib, _dims(), K=FAKE_MIS) == -2                   # misaligned
+    assert _write(lib, _dims(d=48)) == -3                           # unsupported head width
+    assert _write(lib, _dims(h=300)) == -3                          # hidden too wide
+    assert _write(lib, _dims(grid_h=0)) == -1                       # empty grid
+    assert _write(lib, _dims(), ws=None) == -1                      # no workspace
+    assert _write(lib, _dims(), ws=ctypes.c_void_p(0x10010)) == -2  # workspace not 256-aligned
+    assert lib.ttt_read(ctypes.byref(_dims()), None, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert lib.ttt_shortconv2d(ctypes.byref(_dims(d=20)), FAKE, FAKE, FAKE, None) == -3
+    assert lib.ttt_check_status(None, None) == -1
+
+
+def test_workspace_bytes_rejects_bad_dims(lib):
+    assert lib.ttt_workspace_bytes(ctypes.byref(_dims(d=48)), 0) == 0
+    assert lib.ttt_workspace_bytes(ctypes.byref(_dims()), 7) == 0

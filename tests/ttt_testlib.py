@@ -1,0 +1,96 @@
+"""Shared helpers of the parity tests: run the oracle and compare.
+
+Tolerance reading (norm-wise "max relative error"): err(a, ref) =
+max|a - ref| / max|ref|, per tensor and per head.  The GPU path must meet
+O <= 2e-2 and theta* <= 1e-2; the stricter diagnostic on the update itself,
+delta = theta* - theta0, must meet <= 2e-2.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import ttt_oracle as orc
+from test_layer_reconstruction_b200 import inputs as tin
+
+TOL_O = 2e-2
+TOL_THETA = 1e-2
+TOL_DELTA = 2e-2
+
+
+def normwise(a, ref) -> float:
+    a = np.asarray(a, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.max(np.abs(ref))
+    num = np.max(np.abs(a - ref))
+    return float(num / den) if den > 0 else float(num)
+
+
+def dims_of(cfg: tin.LayerConfig) -> orc.Dims:
+    return orc.Dims(cfg.n_views, cfg.grid_h, cfg.grid_w, cfg.n_special)
+
+
+def bf16_inputs(inp):
+    """The GPU path takes bf16 token tensors; the oracle parity run gets the same rounded values."""
+    out = dict(inp)
+    for k in ("Q", "K", "V"):
+        out[k] = tin.bf16_round(inp[k])
+    return out
+
+
+def to_device(inp, device="cuda"):
+    d = {k: inp[k].to(device=device, dtype=torch.bfloat16).contiguous() for k in ("Q", "K", "V") if k in inp}
+    if "conv_w" in inp:
+        d["conv_w"] = inp["conv_w"].to(device=device, dtype=torch.float32).contiguous()
+    if "W1" in inp:
+        d["theta"] = tin.pack_theta(inp["W1"], inp["W3"], inp["W2"]).to(device)
+    return d
+
+
+def oracle_layer(cfg: tin.LayerConfig, inp, heads=None, steps=None, lr=None):
+    """Oracle (float64) over the selected heads; returns dict of per-head arrays."""
+    heads = list(range(cfg.heads)) if heads is None else list(heads)
+    steps = cfg.steps if steps is None else steps
+    lr = cfg.lr if lr is None else lr
+    n, H, d = inp["K"].shape
+    res = {"W1": {}, "W3": {}, "W2": {}, "O": {}, "losses": {}}
+    dims = dims_of(cfg)
+    for hd in heads:
+        ch = slice(hd * d, (hd + 1) * d)
+        V = inp["V"][:, hd].double().numpy()
+        Vp = orc.shortconv2d(V, inp["conv_w"][ch].double().numpy(), dims)
+        th0 = (inp["W1"][hd].double().numpy(), inp["W3"][hd].double().numpy(), inp["W2"][hd].double().numpy())
+        th, ls = orc.sgd_write(inp["K"][:, hd].double().numpy(), Vp, th0, lr, steps)
+        res["W1"][hd], res["W3"][hd], res["W2"][hd] = th
+        res["O"][hd] = orc.read(inp["Q"][:, hd].double().numpy(), *th)
+        res["losses"][hd] = ls
+    return res
+
+
+def compare_theta(cfg, inp, theta_gpu: torch.Tensor, ref, heads=None):
+    """Return worst (theta err, delta err) over heads and the three matrices."""
+    W1g, W3g, W2g = tin.unpack_theta(theta_gpu.detach().cpu(), cfg.heads, cfg.d, cfg.h)
+    gpu = {"W1": W1g, "W3": W3g, "W2": W2g}
+    heads = list(ref["W1"].keys()) if heads is None else heads
+    worst_t, worst_d = 0.0, 0.0
+    for hd in heads:
+        for name in ("W1", "W3", "W2"):
+            g = gpu[name][hd].double().numpy()
+            r = ref[name][hd]
+            t0 = inp[name][hd].double().numpy()
+            worst_t = max(worst_t, normwise(g, r))
+            worst_d = max(worst_d, normwise(g - t0, r - t0))
+    return worst_t, worst_d
+
+
+def compare_O(O_gpu: torch.Tensor, ref, heads=None, rows=None):
+    heads = list(ref["O"].keys()) if heads is None else heads
+    Og = O_gpu.detach().float().cpu()
+    worst = 0.0
+    for hd in heads:
+        r = ref["O"][hd]
+        g = Og[:, hd].double().numpy()
+        if rows is not None:
+            r, g = r[rows], g[rows]
+        worst = max(worst, normwise(g, r))
+    return worst
