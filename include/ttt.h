@@ -119,6 +119,25 @@ int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t*
                    const float* theta0_host, float lr, int steps, float* theta_out_host,
                    uint16_t* O_host, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ttt_read for callers that cannot allocate device memory — for example code
+ * running under an allocator that forbids new device allocations, or a host
+ * that has already handed all device memory to a pool it does not control.
+ * The paper has no counterpart of this entry point; it is a packaging
+ * convenience.  It takes no workspace: its scratch (the status word and the
+ * bf16 fast-weight images) lives in a fixed array of TTT_NOALLOC_SCRATCH_BYTES
+ * bytes that is part of the library, which every GPU that loads the library
+ * holds until the process exits.  Shapes whose scratch would exceed it
+ * (ttt_workspace_bytes(dims, TTT_OP_READ) > TTT_NOALLOC_SCRATCH_BYTES) return
+ * TTT_EWORKSPACE.  The first call on each device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: calls that may overlap on the GPU (other streams, other threads)
+ * race and must be serialised by the caller.  Allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine. */
+#define TTT_NOALLOC_SCRATCH_BYTES (4u << 20)
+int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O,
+                     void* stream);
+
 /* Synchronises `stream`, then reads the device status word of `workspace`:
  * TTT_OK, TTT_EDEVICE if a kernel recorded a fault (the word is cleared), or
  * TTT_ECUDA. */

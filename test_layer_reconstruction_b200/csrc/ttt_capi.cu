@@ -385,9 +385,50 @@ int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) 
   return launch_fwd<false>(s, tq, tq, fp, c.g.fwd, c.st);
 }
 
+// ------------------------------------------------------------------ fixed scratch
+// Scratch of ttt_read_noalloc.  In host code `g_noalloc_scratch` is only a
+// host-side stand-in for the symbol; kernels receive the device address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[TTT_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current); nullptr on failure.
+uint8_t* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return static_cast<uint8_t*>(addr[dev]);
+}
+
 }  // namespace
 
 extern "C" {
+
+int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O, void* stream) {
+  if (!Q || !theta || !O) return TTT_EINVAL;
+  if (!aligned(Q) || !aligned(theta) || !aligned(O)) return TTT_EALIGN;
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != TTT_OK) return rc;
+  const int sms = num_sms();
+  if (sms <= 0) return TTT_ECUDA;
+  if (ws_layout(s, grids_for(s, sms), TTT_OP_READ).total > TTT_NOALLOC_SCRATCH_BYTES) return TTT_EWORKSPACE;
+  uint8_t* scratch = noalloc_scratch();
+  if (!scratch) return TTT_ECUDA;
+  Call c;
+  rc = prepare(dims, TTT_OP_READ, scratch, TTT_NOALLOC_SCRATCH_BYTES, stream, &c);
+  if (rc != TTT_OK) return rc;
+  return run_read(c, Q, theta, O);
+}
 
 size_t ttt_workspace_bytes(const ttt_dims* dims, int op) {
   Shape s;

@@ -23,7 +23,7 @@ __all__ = [
 OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
 EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
                     "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
-                    "ttt_profile_stop", "ttt_kernel_name")
+                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc")
 KERNEL_KINDS = 6
 
 
@@ -85,6 +85,8 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_check_status.argtypes = [P, P]
     lib.ttt_status_str.argtypes = [I]
     lib.ttt_status_str.restype = ctypes.c_char_p
+    lib.ttt_read_noalloc.argtypes = [DP, P, P, P, P]
+    lib.ttt_read_noalloc.restype = I
     lib.ttt_profile_start.argtypes = []
     lib.ttt_profile_stop.argtypes = [ctypes.POINTER(KernelTimes)]
     lib.ttt_kernel_name.argtypes = [I]
