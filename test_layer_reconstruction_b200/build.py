@@ -29,13 +29,17 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the CUDA sources into libttt.so next to this file; return its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str = None, defines=()) -> str:
+    """Compile the CUDA sources into libttt.so next to this file (or `out`); return its path.
+
+    `defines` adds -D flags, e.g. ("TTT_TRACE",) for the per-phase clock trace build."""
+    out = out or LIB
+    if out == LIB and not defines and not force and not _stale():
         return LIB
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
-           "-Xcompiler", "-fPIC", "-shared", "-o", LIB + ".tmp",
+           "-Xcompiler", "-fPIC", "-shared", "-o", out + ".tmp",
            "-I", os.path.join(ROOT, "include")]
+    cmd += [f"-D{d}" for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
@@ -44,8 +48,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

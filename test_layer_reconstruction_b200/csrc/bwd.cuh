@@ -16,14 +16,14 @@
 // kernel sums the partials of a (head, slice) in CTA order, so the result is
 // deterministic.
 //
-// Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
-// allocator + MMA issuer, warps 2-9 two epilogue warpgroups.  Per tile the
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + sub-chunk MMA
+// issuer, warp 10 dW MMA issuer, warps 2-9 two epilogue warpgroups.  Per tile the
 // slice is walked in 4 sub-chunks of 32 hidden units, each with
 //   Z  = K * [W1 | W3]_sub   (M=128 tokens, N=64, K=d)
 //   dA = E * W2_sub^T        (M=128 tokens, N=32, K=d)
 // in one of 3 TMEM slots; the epilogue writes A, dZ1, dZ3 (bf16) to shared
 // memory and the dW MMAs (M=128 hidden, N=d, K=128 tokens, both operands
-// MN-major) of tile j are issued after the sub-chunk MMAs of tile j+1.
+// MN-major) of a tile go out as soon as that is done.
 #pragma once
 #include "fwd.cuh"
 
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[BB_DZ_EMPTY], 1);
     mbar_init(&bars[BB_ACC_FULL], 1);
     mbar_init(&bars[BB_ACC_EMPTY], 8);
-    mbar_init(&bars[BB_DONE], 1);
+    mbar_init(&bars[BB_DONE], 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -120,17 +120,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      TTT_TR_DECL
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_e);
       long long cur_pair = -1;
+      int head = 0, slice = 0;
       uint32_t wl = 0, j = 0;
-      for (long long it = it0; it < it1; ++it, ++j) {
-        const long long pair = it / p.tiles;
-        const int tile = static_cast<int>(it % p.tiles);
-        const int head = static_cast<int>(pair / p.slices);
-        const int slice = static_cast<int>(pair % p.slices);
+      Cursor pf;
+      pf.init(it0, p.tiles);
+      for (int k = 0; k < kPrefetchAhead && pf.it < it1; ++k, pf.next(p.tiles)) {
+        tma_prefetch_l2_2d(&tm_k, (pf.major / p.slices) * D, pf.tile * kTileM);
+        tma_prefetch_l2_2d(&tm_e, (pf.major / p.slices) * D, pf.tile * kTileM);
+      }
+      Cursor cu;
+      cu.init(it0, p.tiles);
+      for (; cu.it < it1; cu.next(p.tiles), ++j) {
+        const int pair = cu.major;
+        const int tile = cu.tile;
         if (pair != cur_pair) {
+          head = pair / p.slices;
+          slice = pair % p.slices;
+          TTT_TR_LAP(0);
           if (wl > 0 && !mbar_wait(&bars[BB_W_EMPTY], (wl - 1) & 1, ab)) break;
+          TTT_TR_LAP(2);
           mbar_arrive_expect_tx(&bars[BB_W_FULL], L::kW13 + L::kW2);
           const size_t hidp = static_cast<size_t>(p.slices) * 128;
           const __nv_bfloat16* w13 = p.w13_img + (static_cast<size_t>(head) * 2 * hidp + slice * 256) * D;
@@ -141,103 +153,113 @@ __global__ void __launch_bounds__(kThreads, 1)
           cur_pair = pair;
         }
         const int s = j & 1;
+        if (pf.it < it1) {
+          tma_prefetch_l2_2d(&tm_k, (pf.major / p.slices) * D, pf.tile * kTileM);
+          tma_prefetch_l2_2d(&tm_e, (pf.major / p.slices) * D, pf.tile * kTileM);
+          pf.next(p.tiles);
+        }
+        TTT_TR_LAP(0);
         if (!mbar_wait(&bars[BB_KE_EMPTY + s], ((j >> 1) & 1) ^ 1, ab)) break;
+        TTT_TR_LAP(1);
         mbar_arrive_expect_tx(&bars[BB_KE_FULL + s], 2 * L::kTile);
         tma_load_2d(smem + L::off_k + s * L::kTile, &tm_k, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
         tma_load_2d(smem + L::off_e + s * L::kTile, &tm_e, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
       }
+      TTT_TR_LAP(0);
+      TTT_TR_DUMP(2);
       if (wl > 0) mbar_drain(&bars[BB_W_FULL], (wl - 1) & 1);
       for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) mbar_drain(&bars[BB_KE_FULL + (jj & 1)], (jj >> 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdZ = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t kIdDA = idesc_bf16(128, 32, false, false);
-      constexpr uint32_t kIdW = idesc_bf16(128, D, true, true);
-      const uint32_t w13 = smem_u32(smem + L::off_w13);
-      const uint32_t w2 = smem_u32(smem + L::off_w2);
-      const uint32_t sa = smem_u32(smem + L::off_a);
-      const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
-      const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
-      long long cur_pair = -1;
-      uint32_t wl = 0, j = 0, kc = 0, seg = 0;
-      bool ok = true, pend = false, pend_first = false;
-      uint32_t pend_j = 0;
-      // dW MMAs of tile qj (stage qj % 2); `first` starts a new accumulation.
-      auto issue_dw = [&](uint32_t qj, bool first) -> bool {
-        if (!mbar_wait(&bars[BB_DZ_FULL], qj & 1, ab)) return false;
-        if (first && seg > 0 && !mbar_wait(&bars[BB_ACC_EMPTY], (seg - 1) & 1, ab)) return false;
-        tc_fence_after();
-        const int s = qj & 1;
-        const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
-        const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
-#pragma unroll
-        for (int k = 0; k < kTileM / 16; ++k) {
-          const uint32_t acc = (first && k == 0) ? 0u : 1u;
-          const uint64_t bk = smem_desc(ks + k * 16 * SW, 0, 8 * SW, SW);
-          const uint64_t be = smem_desc(es + k * 16 * SW, 0, 8 * SW, SW);
-          mma_bf16(tbase + kDw, smem_desc(sdz1 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
-          mma_bf16(tbase + kDw + D, smem_desc(sdz3 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
-          mma_bf16(tbase + kDw + 2 * D, smem_desc(sa + k * 2048, 16384, 1024, 128), be, kIdW, acc);
-        }
-        mma_commit(&bars[BB_DZ_EMPTY]);
-        mma_commit(&bars[BB_KE_EMPTY + s]);
-        return true;
-      };
-      bool seg_first = false;
-      for (long long it = it0; it < it1 && ok; ++it, ++j) {
-        const long long pair = it / p.tiles;
-        if (pair != cur_pair) {
-          if (pend) {
-            if (!(ok = issue_dw(pend_j, pend_first))) break;
-            pend = false;
-          }
-          if (cur_pair >= 0) {
-            mma_commit(&bars[BB_ACC_FULL]);   // segment done: epilogue dumps dW
-            mma_commit(&bars[BB_W_EMPTY]);
-            ++seg;
-          }
-          if (!(ok = mbar_wait(&bars[BB_W_FULL], wl & 1, ab))) break;
-          ++wl;
-          cur_pair = pair;
-          seg_first = true;
-        }
-        const int s = j & 1;
-        if (!(ok = mbar_wait(&bars[BB_KE_FULL + s], (j >> 1) & 1, ab))) break;
-        tc_fence_after();
-        const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
-        const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
-        for (int sc = 0; sc < 4; ++sc, ++kc) {
-          const uint32_t slot = kc % 3, use = kc / 3;
-          if (!(ok = mbar_wait(&bars[BB_SL_EMPTY + slot], (use & 1) ^ 1, ab))) break;
-          tc_fence_after();
-          const uint32_t tsl = tbase + slot * kSlot;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            mma_bf16(tsl, smem_desc(ks + 32 * k, 0, 8 * SW, SW), smem_desc(w13 + 64 * sc * SW + 32 * k, 0, 8 * SW, SW),
-                     kIdZ, k > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            mma_bf16(tsl + 64, smem_desc(es + 32 * k, 0, 8 * SW, SW), smem_desc(w2 + 32 * sc * SW + 32 * k, 0, 8 * SW, SW),
-                     kIdDA, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars[BB_SL_FULL + slot]);
-        }
-        if (!ok) break;
-        if (pend && !(ok = issue_dw(pend_j, pend_first))) break;
-        pend = true;
-        pend_j = j;
-        pend_first = seg_first;
-        seg_first = false;
+    // ------------------------------------------------------------ sub-chunk issuer
+    // Z = K * [W1 | W3]_sub and dA = E * W2_sub^T into one of 3 TMEM slots.
+    constexpr uint32_t kIdZ = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t kIdDA = idesc_bf16(128, 32, false, false);
+    const uint32_t w13 = smem_u32(smem + L::off_w13);
+    const uint32_t w2 = smem_u32(smem + L::off_w2);
+    TTT_TR_DECL
+    Cursor sc;
+    sc.init(it0, p.tiles);
+    int cur_pair = -1;
+    uint32_t sj = 0, kc = 0, wl = 0;
+    bool ok = true;
+    for (; sc.it < it1 && ok; sc.next(p.tiles), ++sj) {
+      if (sc.major != cur_pair) {
+        if (cur_pair >= 0) mma_commit_warp(&bars[BB_W_EMPTY]);
+        if (!(ok = mbar_wait_warp(&bars[BB_W_FULL], wl & 1, ab))) break;
+        ++wl;
+        cur_pair = sc.major;
       }
-      if (ok && pend) ok = issue_dw(pend_j, pend_first);
-      if (ok && cur_pair >= 0) mma_commit(&bars[BB_ACC_FULL]);
-      mma_commit(&bars[BB_DONE]);
-      mbar_drain(&bars[BB_DONE], 0);
+      const int s = sj & 1;
+      TTT_TR_LAP(0);
+      if (!(ok = mbar_wait_warp(&bars[BB_KE_FULL + s], (sj >> 1) & 1, ab))) break;
+      TTT_TR_LAP(1);
+      const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
+      const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
+      for (int ssc = 0; ssc < 4; ++ssc, ++kc) {
+        const uint32_t slot = kc % 3, use = kc / 3;
+        TTT_TR_LAP(0);
+        if (!(ok = mbar_wait_warp(&bars[BB_SL_EMPTY + slot], (use & 1) ^ 1, ab))) break;
+        TTT_TR_LAP(2);
+        tc_fence_after();
+        const uint32_t tsl = tbase + slot * kSlot;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_bf16_warp(tsl, smem_desc(ks + 32 * k, 0, 8 * SW, SW),
+                        smem_desc(w13 + 64 * ssc * SW + 32 * k, 0, 8 * SW, SW), kIdZ, k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_bf16_warp(tsl + 64, smem_desc(es + 32 * k, 0, 8 * SW, SW),
+                        smem_desc(w2 + 32 * ssc * SW + 32 * k, 0, 8 * SW, SW), kIdDA, k > 0 ? 1u : 0u);
+        mma_commit_warp(&bars[BB_SL_FULL + slot]);
+        TTT_TR_LAP(3);
+      }
     }
-  } else {
+    TTT_TR_DUMP(2);
+    mma_commit_warp(&bars[BB_DONE]);
+    mbar_drain(&bars[BB_DONE], 0);
+  } else if (warp == kYWarp) {
+    // ------------------------------------------------------------ dW issuer
+    // dW1^T += dZ1^T K, dW3^T += dZ3^T K, dW2 += A^T E once the epilogue has
+    // written A, dZ1, dZ3 of the tile.  This warp's commit releases the K/E
+    // stage: the tile's sub-chunk MMAs completed before the epilogue could
+    // write its dZ, so every reader of the stage is done.
+    constexpr uint32_t kIdW = idesc_bf16(128, D, true, true);
+    const uint32_t sa = smem_u32(smem + L::off_a);
+    const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
+    const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
+    Cursor wc;
+    wc.init(it0, p.tiles);
+    uint32_t wj = 0, wseg = 0;
+    bool ok = true;
+    for (; wc.it < it1 && ok; wc.next(p.tiles), ++wj) {
+      const bool first = (wc.it == it0) || wc.tile == 0;
+      const bool last = (wc.it == it1 - 1) || wc.tile == p.tiles - 1;
+      if (!(ok = mbar_wait_warp(&bars[BB_DZ_FULL], wj & 1, ab))) break;
+      if (first && wseg > 0 && !(ok = mbar_wait_warp(&bars[BB_ACC_EMPTY], (wseg - 1) & 1, ab))) break;
+      tc_fence_after();
+      const int s = wj & 1;
+      const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
+      const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
+#pragma unroll
+      for (int k = 0; k < kTileM / 16; ++k) {
+        const uint32_t acc = (first && k == 0) ? 0u : 1u;
+        const uint64_t bk = smem_desc(ks + k * 16 * SW, 0, 8 * SW, SW);
+        const uint64_t be = smem_desc(es + k * 16 * SW, 0, 8 * SW, SW);
+        mma_bf16_warp(tbase + kDw, smem_desc(sdz1 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
+        mma_bf16_warp(tbase + kDw + D, smem_desc(sdz3 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
+        mma_bf16_warp(tbase + kDw + 2 * D, smem_desc(sa + k * 2048, 16384, 1024, 128), be, kIdW, acc);
+      }
+      mma_commit_warp(&bars[BB_DZ_EMPTY]);
+      mma_commit_warp(&bars[BB_KE_EMPTY + s]);
+      if (last) {
+        mma_commit_warp(&bars[BB_ACC_FULL]);   // segment done: the epilogue dumps dW
+        ++wseg;
+      }
+    }
+    mma_commit_warp(&bars[BB_DONE]);
+    mbar_drain(&bars[BB_DONE], 0);
+  } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------ epilogue
     const int g = (warp - 2) >> 2;
     const int q = warp & 3;
@@ -249,10 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t j = 0, seg = 0;
     long long cur_pair = -1;
     bool ok = true;
+    TTT_TR_DECL
 
     // Write dW of the finished segment (pair) to its partial slot.
     auto dump = [&](long long pair) -> bool {
+      TTT_TR_LAP(0);
       if (!mbar_wait(&bars[BB_ACC_FULL], seg & 1, ab)) return false;
+      TTT_TR_LAP(5);
       tc_fence_after();
       const long long first_item = pair * p.tiles;
       const long long contrib = blockIdx.x - owner_cta(first_item, total, gridDim.x);
@@ -272,11 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[BB_ACC_EMPTY]);
       ++seg;
+      TTT_TR_LAP(6);
       return true;
     };
 
-    for (long long it = it0; it < it1 && ok; ++it, ++j) {
-      const long long pair = it / p.tiles;
+    Cursor cu;
+    cu.init(it0, p.tiles);
+    for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
+      const long long pair = cu.major;
       if (pair != cur_pair) {
         if (cur_pair >= 0 && !(ok = dump(cur_pair))) break;
         cur_pair = pair;
@@ -285,7 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sc = g; sc < 4; sc += 2) {
         const uint32_t kc = j * 4 + sc;
         const uint32_t slot = kc % 3, use = kc / 3;
+        TTT_TR_LAP(0);
         if (!(ok = mbar_wait(&bars[BB_SL_FULL + slot], use & 1, ab))) break;
+        TTT_TR_LAP(1);
         tc_fence_after();
         const uint32_t tsl = tbase + slot * kSlot + lane_off;
         uint32_t pa[16], pz1[16], pz3[16];
@@ -318,10 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[BB_SL_EMPTY + slot]);
+        TTT_TR_LAP(2);
         if (!waited_buf) {
           if (!(ok = mbar_wait(&bars[BB_DZ_EMPTY], (j & 1) ^ 1, ab))) break;
           waited_buf = true;
         }
+        TTT_TR_LAP(3);
         // hidden unit (within the slice) sc*32 + 8v + e  ->  atom sc/2, 16-byte chunk (sc%2)*4 + v
         const uint32_t base = (sc >> 1) * 16384u;
 #pragma unroll
@@ -336,8 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[BB_DZ_FULL]);
+      TTT_TR_LAP(4);
     }
     if (ok && cur_pair >= 0) dump(cur_pair);
+    TTT_TR_LAP(0);
+    TTT_TR_DUMP(2);
   }
 
   tc_fence_before();

@@ -12,14 +12,15 @@
 // tile) items.  Warp roles:
 //   warp 0   : TMA producer (weights of the current head by bulk copy, X and
 //              V' tiles by 2-D TMA, two stages each)
-//   warp 1   : TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 1   : TMEM allocator and Z issuer, warp 10: Y issuer (each warp
+//              issues in uniform control flow, one elected lane)
 //   warps 2-9: two epilogue warpgroups
 // Per tile the hidden dimension is walked in chunks of 64 units:
 //   Z = X * [W1 | W3]_chunk      (M=128 tokens, N=128, K=d)   -> TMEM slot c%2
 //   A_chunk = silu(Z1) * Z3      (epilogue WG c%2, bf16, smem)
 //   Y += A_chunk * W2_chunk      (M=128, N=d, K=64)            -> TMEM Y slot
-// The MMA warp issues Z of chunk c+1 before Y of chunk c, so the tensor
-// pipe works while an epilogue warpgroup evaluates the gate.  The Y
+// Z and Y have separate issuing warps, so Z of later chunks goes out while
+// an epilogue warpgroup evaluates the gate of an earlier one.  The Y
 // epilogue of tile j runs (in warpgroup j%2) after that warpgroup's chunks
 // of tile j+1.
 #pragma once
@@ -28,7 +29,9 @@
 namespace ttt {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;        // 11 warps
+constexpr int kYWarp = 10;           // second MMA-issuing warp
+constexpr int kPrefetchAhead = 3;   // items whose tiles the producer prefetches into L2
 
 struct FwdParams {
   const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
@@ -75,6 +78,27 @@ __device__ __forceinline__ void bulk_load_pieces(void* dst, const void* src, uin
   }
 }
 
+// Position in the flattened (major, tile) work space (major = head in the
+// forward kernel, (head, hidden slice) pair in the backward kernel), advanced
+// without integer division: the issuing loops run once per MMA group and a
+// 64-bit division costs hundreds of clocks there.
+struct Cursor {
+  long long it;
+  int major, tile;
+  __device__ __forceinline__ void init(long long i, int tiles) {
+    it = i;
+    major = static_cast<int>(i / tiles);
+    tile = static_cast<int>(i % tiles);
+  }
+  __device__ __forceinline__ void next(int tiles) {
+    ++it;
+    if (++tile == tiles) {
+      tile = 0;
+      ++major;
+    }
+  }
+};
+
 // Bounded wait that ignores the abort flag (used only while draining).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -106,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(&bars[FB_W_FULL], 1);
-    mbar_init(&bars[FB_W_EMPTY], 1);
+    mbar_init(&bars[FB_W_EMPTY], 2);    // released by both issuing warps
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[FB_X_FULL + s], 1);
       mbar_init(&bars[FB_X_EMPTY + s], 1);
@@ -119,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[FB_Y_FULL + s], 1);
       mbar_init(&bars[FB_Y_EMPTY + s], 4);
     }
-    mbar_init(&bars[FB_DONE], 1);
+    mbar_init(&bars[FB_DONE], 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -136,13 +160,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      TTT_TR_DECL
       tma_prefetch_desc(&tm_x);
       if (WRITE) tma_prefetch_desc(&tm_vp);
       int cur_head = -1;
       uint32_t wl = 0, j = 0;
-      for (long long it = it0; it < it1; ++it, ++j) {
-        const int head = static_cast<int>(it / p.tiles);
-        const int tile = static_cast<int>(it % p.tiles);
+      Cursor pf;
+      pf.init(it0, p.tiles);
+      for (int k = 0; k < kPrefetchAhead && pf.it < it1; ++k, pf.next(p.tiles)) {
+        tma_prefetch_l2_2d(&tm_x, pf.major * D, pf.tile * kTileM);
+        if (WRITE) tma_prefetch_l2_2d(&tm_vp, pf.major * D, pf.tile * kTileM);
+      }
+      Cursor cu;
+      cu.init(it0, p.tiles);
+      for (; cu.it < it1; cu.next(p.tiles), ++j) {
+        const int head = cu.major;
+        const int tile = cu.tile;
         if (head != cur_head) {
           if (wl > 0 && !mbar_wait(&bars[FB_W_EMPTY], (wl - 1) & 1, ab)) break;
           mbar_arrive_expect_tx(&bars[FB_W_FULL], L::kW13 + L::kW2);
@@ -155,15 +188,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
+        // Warm L2 with the tiles a few items ahead so the shared-memory loads hit L2.
+        if (pf.it < it1) {
+          tma_prefetch_l2_2d(&tm_x, pf.major * D, pf.tile * kTileM);
+          if (WRITE) tma_prefetch_l2_2d(&tm_vp, pf.major * D, pf.tile * kTileM);
+          pf.next(p.tiles);
+        }
+        TTT_TR_LAP(0);
         if (!mbar_wait(&bars[FB_X_EMPTY + s], ph ^ 1, ab)) break;
+        TTT_TR_LAP(1);
         mbar_arrive_expect_tx(&bars[FB_X_FULL + s], L::kTile);
         tma_load_2d(smem + L::off_x + s * L::kTile, &tm_x, &bars[FB_X_FULL + s], head * D, tile * kTileM);
         if (WRITE) {
+          TTT_TR_LAP(0);
           if (!mbar_wait(&bars[FB_VP_EMPTY + s], ph ^ 1, ab)) break;
+          TTT_TR_LAP(2);
           mbar_arrive_expect_tx(&bars[FB_VP_FULL + s], L::kTile);
           tma_load_2d(smem + L::off_vp + s * L::kTile, &tm_vp, &bars[FB_VP_FULL + s], head * D, tile * kTileM);
         }
       }
+      TTT_TR_LAP(0);
+      TTT_TR_DUMP(WRITE ? 0 : 1);
       // Drain: the last load issued into each barrier has landed before exit.
       if (wl > 0) mbar_drain(&bars[FB_W_FULL], (wl - 1) & 1);
       for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) {
@@ -172,78 +217,87 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdZ = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t kIdY = idesc_bf16(128, D, false, true);
-      const uint32_t w13 = smem_u32(smem + L::off_w13);
-      const uint32_t w2 = smem_u32(smem + L::off_w2);
-      int cur_head = -1;
-      uint32_t wl = 0, j = 0, zc = 0;
-      bool pend = false, ok = true;
-      uint32_t pend_j = 0;
-      int pend_c = 0;
-      // Y += A_chunk * W2_chunk for a chunk whose gate the epilogue has written.
-      auto issue_y = [&](uint32_t qj, int qc) -> bool {
-        const uint32_t ys = qj & 1;
-        if (qc == 0 && !mbar_wait(&bars[FB_Y_EMPTY + ys], ((qj >> 1) & 1) ^ 1, ab)) return false;
-        const int g = qc & 1;
-        const uint32_t u = qj * (NC / 2) + (qc >> 1);
-        if (!mbar_wait(&bars[FB_A_FULL + g], u & 1, ab)) return false;
+    // ------------------------------------------------------------ Z issuer
+    // Z = X * [W1 | W3]_chunk into TMEM slot c % 2 as soon as the slot is free.
+    constexpr uint32_t kIdZ = idesc_bf16(128, 128, false, false);
+    const uint32_t w13 = smem_u32(smem + L::off_w13);
+    TTT_TR_DECL
+    Cursor zc;
+    zc.init(it0, p.tiles);
+    int cur_head = -1;
+    uint32_t zj = 0, zcount = 0, wl = 0;
+    bool ok = true;
+    for (; zc.it < it1 && ok; zc.next(p.tiles), ++zj) {
+      if (zc.major != cur_head) {
+        if (cur_head >= 0) mma_commit_warp(&bars[FB_W_EMPTY]);
+        if (!(ok = mbar_wait_warp(&bars[FB_W_FULL], wl & 1, ab))) break;
+        ++wl;
+        cur_head = zc.major;
+      }
+      const int s = zj & 1;
+      TTT_TR_LAP(0);
+      if (!(ok = mbar_wait_warp(&bars[FB_X_FULL + s], (zj >> 1) & 1, ab))) break;
+      TTT_TR_LAP(1);
+      const uint32_t xa = smem_u32(smem + L::off_x + s * L::kTile);
+      for (int c = 0; c < NC; ++c, ++zcount) {
+        const int zs = c & 1;
+        TTT_TR_LAP(0);
+        if (!(ok = mbar_wait_warp(&bars[FB_Z_EMPTY + zs], ((zcount >> 1) & 1) ^ 1, ab))) break;
+        TTT_TR_LAP(2);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = smem_desc(xa + 32 * k, 0, 8 * SW, SW);
+          const uint64_t bd = smem_desc(w13 + 128 * c * SW + 32 * k, 0, 8 * SW, SW);
+          mma_bf16_warp(tz + zs * 128, ad, bd, kIdZ, k > 0 ? 1u : 0u);
+        }
+        mma_commit_warp(&bars[FB_Z_FULL + zs]);
+        TTT_TR_LAP(3);
+      }
+      if (ok) mma_commit_warp(&bars[FB_X_EMPTY + s]);
+    }
+    TTT_TR_DUMP(WRITE ? 0 : 1);
+    // All issued MMAs have completed before TMEM is released.
+    mma_commit_warp(&bars[FB_DONE]);
+    mbar_drain(&bars[FB_DONE], 0);
+  } else if (warp == kYWarp) {
+    // ------------------------------------------------------------ Y issuer
+    // Y += A_chunk * W2_chunk once the gate of the chunk is in shared memory.
+    constexpr uint32_t kIdY = idesc_bf16(128, D, false, true);
+    const uint32_t w2 = smem_u32(smem + L::off_w2);
+    Cursor yc;
+    yc.init(it0, p.tiles);
+    int cur_head = -1;
+    uint32_t yj = 0, wl = 0;
+    bool ok = true;
+    for (; yc.it < it1 && ok; yc.next(p.tiles), ++yj) {
+      if (yc.major != cur_head) {
+        if (cur_head >= 0) mma_commit_warp(&bars[FB_W_EMPTY]);
+        if (!(ok = mbar_wait_warp(&bars[FB_W_FULL], wl & 1, ab))) break;
+        ++wl;
+        cur_head = yc.major;
+      }
+      const uint32_t ys = yj & 1;
+      if (!(ok = mbar_wait_warp(&bars[FB_Y_EMPTY + ys], ((yj >> 1) & 1) ^ 1, ab))) break;
+      for (int c = 0; c < NC; ++c) {
+        const int g = c & 1;
+        const uint32_t u = yj * (NC / 2) + (c >> 1);
+        if (!(ok = mbar_wait_warp(&bars[FB_A_FULL + g], u & 1, ab))) break;
         tc_fence_after();
         const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint64_t ad = smem_desc(abuf + 32 * k, 0, 1024, 128);
-          const uint64_t bd = smem_desc(w2 + (64 * qc + 16 * k) * SW, HIDP * SW, 8 * SW, SW);
-          mma_bf16(ty + ys * D, ad, bd, kIdY, (qc > 0 || k > 0) ? 1u : 0u);
+          const uint64_t bd = smem_desc(w2 + (64 * c + 16 * k) * SW, HIDP * SW, 8 * SW, SW);
+          mma_bf16_warp(ty + ys * D, ad, bd, kIdY, (c > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(&bars[FB_A_EMPTY + g]);
-        if (qc == NC - 1) mma_commit(&bars[FB_Y_FULL + ys]);
-        return true;
-      };
-      for (long long it = it0; it < it1 && ok; ++it, ++j) {
-        const int head = static_cast<int>(it / p.tiles);
-        if (head != cur_head) {
-          if (pend) {
-            if (!(ok = issue_y(pend_j, pend_c))) break;
-            pend = false;
-          }
-          if (cur_head >= 0) mma_commit(&bars[FB_W_EMPTY]);
-          if (!(ok = mbar_wait(&bars[FB_W_FULL], wl & 1, ab))) break;
-          ++wl;
-          cur_head = head;
-        }
-        const int s = j & 1;
-        if (!(ok = mbar_wait(&bars[FB_X_FULL + s], (j >> 1) & 1, ab))) break;
-        tc_fence_after();
-        const uint32_t xa = smem_u32(smem + L::off_x + s * L::kTile);
-        for (int c = 0; c < NC; ++c) {
-          const int zs = c & 1;
-          const uint32_t use = zc >> 1;
-          if (!(ok = mbar_wait(&bars[FB_Z_EMPTY + zs], (use & 1) ^ 1, ab))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t ad = smem_desc(xa + 32 * k, 0, 8 * SW, SW);
-            const uint64_t bd = smem_desc(w13 + 128 * c * SW + 32 * k, 0, 8 * SW, SW);
-            mma_bf16(tz + zs * 128, ad, bd, kIdZ, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars[FB_Z_FULL + zs]);
-          if (c == NC - 1) mma_commit(&bars[FB_X_EMPTY + s]);
-          ++zc;
-          if (pend && !(ok = issue_y(pend_j, pend_c))) break;
-          pend = true;
-          pend_j = j;
-          pend_c = c;
-        }
+        mma_commit_warp(&bars[FB_A_EMPTY + g]);
       }
-      if (ok && pend) issue_y(pend_j, pend_c);
-      // All issued MMAs have completed before TMEM is released.
-      mma_commit(&bars[FB_DONE]);
-      mbar_drain(&bars[FB_DONE], 0);
+      if (ok) mma_commit_warp(&bars[FB_Y_FULL + ys]);
     }
-  } else {
+    mma_commit_warp(&bars[FB_DONE]);
+    mbar_drain(&bars[FB_DONE], 0);
+  } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------ epilogue
     const int g = (warp - 2) >> 2;          // warpgroup
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
@@ -251,14 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
     uint32_t j = 0, u = 0;
-    long long prev_it = -1;
+    TTT_TR_DECL
 
-    // Y epilogue of tile jj (item `itj`), done by warpgroup jj % 2.
-    auto y_epilogue = [&](uint32_t jj, long long itj) -> bool {
-      const int head = static_cast<int>(itj / p.tiles);
-      const int tile = static_cast<int>(itj % p.tiles);
+    // Y epilogue of tile jj (head, tile), done by warpgroup jj % 2.
+    auto y_epilogue = [&](uint32_t jj, int head, int tile) -> bool {
       const uint32_t ys = jj & 1;
+      TTT_TR_LAP(0);
       if (!mbar_wait(&bars[FB_Y_FULL + ys], (jj >> 1) & 1, ab)) return false;
+      TTT_TR_LAP(5);
       tc_fence_after();
       float y[D];
       const uint32_t yb = ty + ys * D + lane_off;
@@ -303,13 +357,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[ch] = v;
         }
       }
+      TTT_TR_LAP(6);
       return true;
     };
 
     bool ok = true;
-    for (long long it = it0; it < it1 && ok; ++it, ++j) {
+    int prev_head = 0, prev_tile = 0;
+    Cursor cu;
+    cu.init(it0, p.tiles);
+    for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
       for (int c = g; c < NC; c += 2, ++u) {
+        TTT_TR_LAP(0);
         if (!(ok = mbar_wait(&bars[FB_Z_FULL + g], u & 1, ab))) break;
+        TTT_TR_LAP(1);
         tc_fence_after();
         uint32_t apk[32];  // 64 gate values of this row, bf16 pairs
         const uint32_t zb = tz + g * 128 + lane_off;
@@ -333,7 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + g]);
+        TTT_TR_LAP(2);
         if (!(ok = mbar_wait(&bars[FB_A_EMPTY + g], (u & 1) ^ 1, ab))) break;
+        TTT_TR_LAP(3);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch)
           st_shared_v4(abuf + swz(row * 128 + ch * 16, 128), apk[4 * ch], apk[4 * ch + 1], apk[4 * ch + 2],
@@ -341,12 +403,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[FB_A_FULL + g]);
+        TTT_TR_LAP(4);
       }
       if (!ok) break;
-      if (j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) ok = y_epilogue(j - 1, prev_it);
-      prev_it = it;
+      if (j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) ok = y_epilogue(j - 1, prev_head, prev_tile);
+      prev_head = cu.major;
+      prev_tile = cu.tile;
     }
-    if (ok && j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) y_epilogue(j - 1, prev_it);
+    if (ok && j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) y_epilogue(j - 1, prev_head, prev_tile);
+    TTT_TR_LAP(0);
+    TTT_TR_DUMP(WRITE ? 0 : 1);
   }
 
   tc_fence_before();

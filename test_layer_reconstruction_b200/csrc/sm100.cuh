@@ -50,6 +50,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe: true if the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Per-CTA abort flag in shared memory plus the global status word.  A wait
 // that runs out records the fault, raises the CTA's abort flag and returns
 // false; every role then leaves its loop and the CTA tears down normally.
@@ -99,6 +112,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// Prefetch a 2-D tile into L2 (no shared memory, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 // 2-D tile store shared -> global (rows outside the tensor are clipped).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -146,6 +165,52 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Warp-collective forms: the whole warp runs the issuing code in uniform
+// control flow (so descriptors stay in uniform registers) and one elected
+// lane issues.  Issuing from a single divergent lane instead costs ~120 SM
+// clocks per MMA on B200, far more than an N <= 128 MMA takes to execute.
+__device__ __forceinline__ void mma_bf16_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// A operand from tensor memory (`a_tmem`: its first column), B from shared memory.
+__device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// Warp-uniform barrier probe: true once every lane has observed the phase
+// completed (so whichever lane is elected has itself acquired it).
+__device__ __forceinline__ bool mbar_test_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_test(bar, parity));
+}
+
+// Warp-uniform bounded wait: every lane waits (hardware-suspended try_wait)
+// and the warp proceeds together.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  const bool ok = mbar_wait(bar, parity, ab);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -209,6 +274,47 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 __host__ __device__ constexpr uint32_t swz(uint32_t off, int sw) {
   return off ^ (((off >> 7) & static_cast<uint32_t>(sw / 16 - 1)) << 4);
 }
+
+// ----------------------------------------------------------------- tracing
+// Built with -DTTT_TRACE, every warp accumulates SM clocks per pipeline phase
+// (index 0..7, meaning fixed per role) and adds them to g_ttt_trace at exit;
+// the host reads them with ttt_trace_read.  Off by default: the macros expand
+// to nothing.
+#ifdef TTT_TRACE
+constexpr int kTraceKernels = 3, kTraceWarps = 11, kTraceSlots = 8;
+// Defined here: the library is a single translation unit.
+__device__ unsigned long long g_ttt_trace[kTraceKernels * kTraceWarps * kTraceSlots];
+struct Tracer {
+  unsigned long long acc[kTraceSlots];
+  long long t;
+  __device__ __forceinline__ void start() {
+#pragma unroll
+    for (int i = 0; i < kTraceSlots; ++i) acc[i] = 0;
+    t = clock64();
+  }
+  __device__ __forceinline__ void lap(int i) {
+    const long long now = clock64();
+    acc[i] += static_cast<unsigned long long>(now - t);
+    t = now;
+  }
+  __device__ __forceinline__ void dump(int kernel, int warp, int lane) {
+    if (lane != 0) return;
+    for (int i = 0; i < kTraceSlots; ++i)
+      atomicAdd(&g_ttt_trace[(kernel * kTraceWarps + warp) * kTraceSlots + i], acc[i]);
+  }
+};
+#define TTT_TR_DECL \
+  ttt::Tracer tr_;   \
+  tr_.start();
+#define TTT_TR_LAP(i) tr_.lap(i)
+#define TTT_TR_COUNT(i) (tr_.acc[i] += 1)
+#define TTT_TR_DUMP(k) tr_.dump((k), threadIdx.x >> 5, threadIdx.x & 31)
+#else
+#define TTT_TR_DECL
+#define TTT_TR_LAP(i)
+#define TTT_TR_COUNT(i)
+#define TTT_TR_DUMP(k)
+#endif
 
 // ----------------------------------------------------------------- math
 __device__ __forceinline__ float tanh_approx(float x) {

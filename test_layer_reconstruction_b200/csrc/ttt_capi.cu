@@ -413,6 +413,19 @@ uint8_t* noalloc_scratch() {
 
 extern "C" {
 
+#ifdef TTT_TRACE
+// Trace builds only: copy out (and with reset != 0, clear) the per-warp phase clocks.
+int ttt_trace_read(unsigned long long* out, int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return TTT_ECUDA;
+  if (cudaMemcpyFromSymbol(out, ttt::g_ttt_trace, sizeof(ttt::g_ttt_trace)) != cudaSuccess) return TTT_ECUDA;
+  if (reset) {
+    static unsigned long long zeros[ttt::kTraceKernels * ttt::kTraceWarps * ttt::kTraceSlots] = {};
+    if (cudaMemcpyToSymbol(ttt::g_ttt_trace, zeros, sizeof(zeros)) != cudaSuccess) return TTT_ECUDA;
+  }
+  return TTT_OK;
+}
+#endif
+
 int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O, void* stream) {
   if (!Q || !theta || !O) return TTT_EINVAL;
   if (!aligned(Q) || !aligned(theta) || !aligned(O)) return TTT_EALIGN;
