@@ -11,9 +11,10 @@
 //   dZ1 = dA * Z3 * S * (1 + Z1 (1 - S)),  dZ3 = dA * Z1 * S,  A = Z1 S Z3
 //   dW1^T += dZ1^T K,  dW3^T += dZ3^T K,  dW2 += A^T E
 // CTA work = (head, 128-wide slice of the hidden units, contiguous range of
-// 128-token tiles); dW for the slice stays in TMEM for the whole range and is
-// written once per (head, slice) segment to a partial buffer.  The update
-// kernel sums the partials of a (head, slice) in CTA order, so the result is
+// 128-token tiles); the CTAs of one group share the tile range, one slice
+// each.  dW for the slice stays in TMEM for the whole range and is written
+// once per (head, slice) segment to a partial buffer.  The update kernel sums
+// the partials of a (head, slice) in group order, so the result is
 // deterministic.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + sub-chunk MMA
@@ -29,10 +30,13 @@
 
 namespace ttt {
 
+constexpr int kBwdThreads = 352;    // 11 warps: 0 producer, 1 sub-chunk issuer, 2-9 epilogue, 10 dW issuer
+constexpr int kBwdDwWarp = 10;
+
 struct BwdParams {
   const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
   const __nv_bfloat16* w2_img;   // per head: HIDP rows of D bf16 (sw-swizzled)
-  float* partials;               // [pairs][max_contrib][3][128][D] f32
+  float* partials;               // [head*slices+slice][max_contrib][3][128][D] f32
   int n, heads, tiles, slices;   // slices = HIDP / 128
   int max_contrib;
   unsigned int* status;
@@ -63,14 +67,14 @@ enum BwdBar {
   BB_DZ_FULL = 12, BB_DZ_EMPTY = 13, BB_ACC_FULL = 14, BB_ACC_EMPTY = 15, BB_DONE = 16
 };
 
-// CTA that owns flattened work item i under the static partition
-// [floor(c*N/G), floor((c+1)*N/G)).
+// Group (of CTAs) that owns flattened (head, tile) item i under the static
+// partition [floor(g*N/G), floor((g+1)*N/G)).
 __host__ __device__ inline long long owner_cta(long long i, long long n_items, long long grid) {
   return ((i + 1) * grid - 1) / n_items;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_e,
                const BwdParams p) {
   using L = BwdLayout<D>;
@@ -85,9 +89,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Abort ab{abort_flag, p.status};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const long long total = static_cast<long long>(p.heads) * p.slices * p.tiles;
-  const long long it0 = total * blockIdx.x / gridDim.x;
-  const long long it1 = total * (blockIdx.x + 1) / gridDim.x;
+  // CTAs come in groups of `slices`: CTA group*slices + s handles hidden slice s
+  // of the group's (head, tile) range, so the CTAs of a group read the same K/E
+  // tiles at about the same time and all but the first find them in L2.
+  const int slice_id = blockIdx.x % p.slices;
+  const int group = blockIdx.x / p.slices;
+  const int groups = gridDim.x / p.slices;
+  const long long total = static_cast<long long>(p.heads) * p.tiles;
+  const long long it0 = total * group / groups;
+  const long long it1 = total * (group + 1) / groups;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -129,17 +139,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       Cursor pf;
       pf.init(it0, p.tiles);
       for (int k = 0; k < kPrefetchAhead && pf.it < it1; ++k, pf.next(p.tiles)) {
-        tma_prefetch_l2_2d(&tm_k, (pf.major / p.slices) * D, pf.tile * kTileM);
-        tma_prefetch_l2_2d(&tm_e, (pf.major / p.slices) * D, pf.tile * kTileM);
+        tma_prefetch_l2_2d(&tm_k, pf.major * D, pf.tile * kTileM);
+        tma_prefetch_l2_2d(&tm_e, pf.major * D, pf.tile * kTileM);
       }
       Cursor cu;
       cu.init(it0, p.tiles);
       for (; cu.it < it1; cu.next(p.tiles), ++j) {
-        const int pair = cu.major;
+        const int pair = cu.major * p.slices + slice_id;
         const int tile = cu.tile;
         if (pair != cur_pair) {
-          head = pair / p.slices;
-          slice = pair % p.slices;
+          head = cu.major;
+          slice = slice_id;
           TTT_TR_LAP(0);
           if (wl > 0 && !mbar_wait(&bars[BB_W_EMPTY], (wl - 1) & 1, ab)) break;
           TTT_TR_LAP(2);
@@ -154,8 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int s = j & 1;
         if (pf.it < it1) {
-          tma_prefetch_l2_2d(&tm_k, (pf.major / p.slices) * D, pf.tile * kTileM);
-          tma_prefetch_l2_2d(&tm_e, (pf.major / p.slices) * D, pf.tile * kTileM);
+          tma_prefetch_l2_2d(&tm_k, pf.major * D, pf.tile * kTileM);
+          tma_prefetch_l2_2d(&tm_e, pf.major * D, pf.tile * kTileM);
           pf.next(p.tiles);
         }
         TTT_TR_LAP(0);
@@ -218,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     TTT_TR_DUMP(2);
     mma_commit_warp(&bars[BB_DONE]);
     mbar_drain(&bars[BB_DONE], 0);
-  } else if (warp == kYWarp) {
+  } else if (warp == kBwdDwWarp) {
     // ------------------------------------------------------------ dW issuer
     // dW1^T += dZ1^T K, dW3^T += dZ3^T K, dW2 += A^T E once the epilogue has
     // written A, dZ1, dZ3 of the tile.  This warp's commit releases the K/E
@@ -279,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars[BB_ACC_FULL], seg & 1, ab)) return false;
       TTT_TR_LAP(5);
       tc_fence_after();
-      const long long first_item = pair * p.tiles;
-      const long long contrib = blockIdx.x - owner_cta(first_item, total, gridDim.x);
+      const long long first_item = (pair / p.slices) * static_cast<long long>(p.tiles);
+      const long long contrib = group - owner_cta(first_item, total, groups);
       float* dst = p.partials + (static_cast<size_t>(pair) * p.max_contrib + contrib) * (3u * 128u * D);
       for (int grp = g; grp < 3 * D / 16; grp += 2) {
         uint32_t r[16];
@@ -304,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor cu;
     cu.init(it0, p.tiles);
     for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
-      const long long pair = cu.major;
+      const long long pair = static_cast<long long>(cu.major) * p.slices + slice_id;
       if (pair != cur_pair) {
         if (cur_pair >= 0 && !(ok = dump(cur_pair))) break;
         cur_pair = pair;
@@ -318,36 +328,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         TTT_TR_LAP(1);
         tc_fence_after();
         const uint32_t tsl = tbase + slot * kSlot + lane_off;
-        uint32_t pa[16], pz1[16], pz3[16];
+        // Load the whole sub-chunk (Z1, Z3, dA), return the slot to the MMA
+        // issuer at once, then compute from registers.
+        uint32_t zz1[2][16], zz3[2][16], zda[2][16];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t z1[16], z3[16], da[16];
-          tmem_ld16(tsl + half * 16, z1);
-          tmem_ld16(tsl + 32 + half * 16, z3);
-          tmem_ld16(tsl + 64 + half * 16, da);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            float av[2], d1[2], d3[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const float x1 = __uint_as_float(z1[i + t]), x3 = __uint_as_float(z3[i + t]);
-              const float dav = __uint_as_float(da[i + t]);
-              const float sg = sigmoid_fast(x1);
-              const float silu = x1 * sg;
-              const float tt = x3 * sg;
-              av[t] = silu * x3;
-              d1[t] = dav * fmaf(tt * x1, 1.0f - sg, tt);
-              d3[t] = dav * silu;
-            }
-            pa[half * 8 + i / 2] = pack_bf16x2(av[0], av[1]);
-            pz1[half * 8 + i / 2] = pack_bf16x2(d1[0], d1[1]);
-            pz3[half * 8 + i / 2] = pack_bf16x2(d3[0], d3[1]);
-          }
+          tmem_ld16(tsl + half * 16, zz1[half]);
+          tmem_ld16(tsl + 32 + half * 16, zz3[half]);
+          tmem_ld16(tsl + 64 + half * 16, zda[half]);
         }
+        tmem_wait_ld();
+        TTT_TR_LAP(7);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[BB_SL_EMPTY + slot]);
+        uint32_t pa[16], pz1[16], pz3[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t (&z1)[16] = zz1[half];
+          const uint32_t (&z3)[16] = zz3[half];
+          const uint32_t (&da)[16] = zda[half];
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            // Packed bf16 arithmetic on two hidden units (the outputs are the
+            // bf16 operands of the dW MMAs): with s = sigmoid(z1) =
+            // (1 + tanh(z1/2))/2, silu = z1 s, A = silu z3, and
+            // d silu/dz1 = s (1 + z1 (1 - s)):
+            //   dZ1 = dA * (z3 s + z3 s * z1 (1 - s)),  dZ3 = dA * silu.
+            const uint32_t b1 = pack_bf16x2(__uint_as_float(z1[i]), __uint_as_float(z1[i + 1]));
+            const uint32_t b3 = pack_bf16x2(__uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
+            const uint32_t bd = pack_bf16x2(__uint_as_float(da[i]), __uint_as_float(da[i + 1]));
+            const uint32_t sg = bfma2(btanh2(bmul2(b1, kBf2Half)), kBf2Half, kBf2Half);
+            const uint32_t silu = bmul2(b1, sg);
+            const uint32_t tt = bmul2(b3, sg);
+            const uint32_t w = bmul2(b1, bfma2(sg, kBf2NegOne, kBf2One));
+            pa[half * 8 + i / 2] = bmul2(silu, b3);
+            pz1[half * 8 + i / 2] = bmul2(bd, bfma2(tt, w, tt));
+            pz3[half * 8 + i / 2] = bmul2(bd, silu);
+          }
+        }
         TTT_TR_LAP(2);
         if (!waited_buf) {
           if (!(ok = mbar_wait(&bars[BB_DZ_EMPTY], (j & 1) ^ 1, ab))) break;

@@ -11,31 +11,37 @@
 // One persistent CTA per SM walks a contiguous range of (head, 128-token
 // tile) items.  Warp roles:
 //   warp 0   : TMA producer (weights of the current head by bulk copy, X and
-//              V' tiles by 2-D TMA, two stages each)
-//   warp 1   : TMEM allocator and Z issuer, warp 10: Y issuer (each warp
-//              issues in uniform control flow, one elected lane)
-//   warps 2-9: two epilogue warpgroups
+//              V' tiles by 2-D TMA, two stages each, L2 prefetch ahead)
+//   warp 1   : TMEM allocator and Z issuer
+//   warp 2   : Y issuer (warp 3 idles)
+//   warps 4-19: four epilogue warpgroups; warpgroups 2p and 2p+1 share the
+//              chunks c with c % 2 == p, one 32-unit half of the chunk each
+// Both issuers run in uniform control flow and issue from one elected lane.
 // Per tile the hidden dimension is walked in chunks of 64 units:
-//   Z = X * [W1 | W3]_chunk      (M=128 tokens, N=128, K=d)   -> TMEM slot c%2
-//   A_chunk = silu(Z1) * Z3      (epilogue WG c%2, bf16, smem)
-//   Y += A_chunk * W2_chunk      (M=128, N=d, K=64)            -> TMEM Y slot
-// Z and Y have separate issuing warps, so Z of later chunks goes out while
-// an epilogue warpgroup evaluates the gate of an earlier one.  The Y
-// epilogue of tile j runs (in warpgroup j%2) after that warpgroup's chunks
-// of tile j+1.
+//   Z = X * [W1 | W3]_chunk        (M=128 tokens, N=128, K=d, A and B in smem)
+//                                    -> TMEM Z slot c % 2
+//   gate = silu(Z1) * Z3           (epilogue warpgroups 2(c%2), 2(c%2)+1, packed
+//                                    f16 arithmetic) -> TMEM gate slot c % 2
+//   Y += gate * W2_chunk           (M=128, N=d, K=64, A from TMEM, B = f16 W2
+//                                    image in smem) -> TMEM Y slot j % 2
+// Keeping the gate in tensor memory avoids a shared-memory round trip and
+// lets the N=d MMA run at full rate.  The Y epilogue of tile j runs in the
+// warpgroup pair j % 2 (one half of the columns each) after that pair's
+// chunks of tile j+1.
 #pragma once
 #include "sm100.cuh"
 
 namespace ttt {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 352;        // 11 warps
-constexpr int kYWarp = 10;           // second MMA-issuing warp
-constexpr int kPrefetchAhead = 3;   // items whose tiles the producer prefetches into L2
+constexpr int kThreads = 640;        // 20 warps: 0 producer, 1 Z issuer, 2 Y issuer, 3 idle, 4-19 epilogue
+constexpr int kYWarp = 2;            // second MMA-issuing warp
+constexpr int kEpiWarp0 = 4;         // first epilogue warp (4 warpgroups of 4)
+constexpr int kPrefetchAhead = 3;    // items whose tiles the producer prefetches into L2
 
 struct FwdParams {
   const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
-  const __nv_bfloat16* w2_img;   // per head: HIDP rows of D bf16 (sw-swizzled)
+  const __half* w2_img;          // per head: HIDP rows of D f16 (sw-swizzled)
   __nv_bfloat16* out;            // [n][heads][D]
   int n, heads, tiles;
   unsigned int* status;
@@ -47,17 +53,20 @@ struct FwdLayout {
   static constexpr uint32_t kW13 = 2u * HIDP * D * 2;
   static constexpr uint32_t kW2 = 1u * HIDP * D * 2;
   static constexpr uint32_t kTile = 1u * kTileM * D * 2;
-  static constexpr uint32_t kA = kTileM * 64 * 2;
   static constexpr uint32_t off_w13 = 0;
   static constexpr uint32_t off_w2 = off_w13 + kW13;
   static constexpr uint32_t off_x = off_w2 + kW2;
   static constexpr uint32_t off_vp = off_x + 2 * kTile;
-  static constexpr uint32_t off_a = off_vp + 2 * kTile;
-  static constexpr uint32_t off_bar = off_a + 2 * kA;
+  static constexpr uint32_t off_bar = off_vp + 2 * kTile;
   static constexpr int kNumBars = 24;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
-  static_assert(off_x % 1024 == 0 && off_vp % 1024 == 0 && off_a % 1024 == 0, "1 KiB alignment");
+  static_assert(off_x % 1024 == 0 && off_vp % 1024 == 0, "1 KiB alignment");
 };
+
+// TMEM columns
+constexpr uint32_t kFwdZCols = 0;      // 2 Z slots x 128
+constexpr uint32_t kFwdGateCols = 256; // 2 gate slots x 32 (64 f16 per row)
+constexpr uint32_t kFwdYCols = 320;    // 2 Y slots x D
 
 // barrier indices
 enum FwdBar {
@@ -107,6 +116,16 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Gate of two hidden units in packed f16: silu(z1) * z3 with
+// sigmoid(z) = (1 + tanh(z/2)) / 2.
+__device__ __forceinline__ uint32_t gate_f16x2(float z1a, float z1b, float z3a, float z3b) {
+  const uint32_t h1 = pack_f16x2(z1a, z1b);
+  const uint32_t h3 = pack_f16x2(z3a, z3b);
+  const uint32_t t = htanh2(hmul2(h1, kHalf2Half));
+  const uint32_t s = hfma2(t, kHalf2Half, kHalf2Half);
+  return hmul2(hmul2(h1, s), h3);
+}
+
 template <int D, int HIDP, bool WRITE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_vp,
@@ -135,13 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[FB_X_FULL + s], 1);
       mbar_init(&bars[FB_X_EMPTY + s], 1);
       mbar_init(&bars[FB_VP_FULL + s], 1);
-      mbar_init(&bars[FB_VP_EMPTY + s], 4);
+      mbar_init(&bars[FB_VP_EMPTY + s], 8);
       mbar_init(&bars[FB_Z_FULL + s], 1);
-      mbar_init(&bars[FB_Z_EMPTY + s], 4);
-      mbar_init(&bars[FB_A_FULL + s], 4);
+      mbar_init(&bars[FB_Z_EMPTY + s], 8);
+      mbar_init(&bars[FB_A_FULL + s], 8);
       mbar_init(&bars[FB_A_EMPTY + s], 1);
       mbar_init(&bars[FB_Y_FULL + s], 1);
-      mbar_init(&bars[FB_Y_EMPTY + s], 4);
+      mbar_init(&bars[FB_Y_EMPTY + s], 8);
     }
     mbar_init(&bars[FB_DONE], 2);
     fence_mbar_init();
@@ -154,8 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tz = tbase;          // 2 Z slots x 128 columns
-  const uint32_t ty = tbase + 256;    // 2 Y slots x D columns
+  const uint32_t tz = tbase + kFwdZCols;
+  const uint32_t tg = tbase + kFwdGateCols;
+  const uint32_t ty = tbase + kFwdYCols;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -262,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_drain(&bars[FB_DONE], 0);
   } else if (warp == kYWarp) {
     // ------------------------------------------------------------ Y issuer
-    // Y += A_chunk * W2_chunk once the gate of the chunk is in shared memory.
-    constexpr uint32_t kIdY = idesc_bf16(128, D, false, true);
+    // Y += gate_chunk * W2_chunk once the gate of the chunk is in TMEM.
+    constexpr uint32_t kIdY = idesc_f16(128, D, false, true);
     const uint32_t w2 = smem_u32(smem + L::off_w2);
     Cursor yc;
     yc.init(it0, p.tiles);
@@ -284,12 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t u = yj * (NC / 2) + (c >> 1);
         if (!(ok = mbar_wait_warp(&bars[FB_A_FULL + g], u & 1, ab))) break;
         tc_fence_after();
-        const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = smem_desc(abuf + 32 * k, 0, 1024, 128);
           const uint64_t bd = smem_desc(w2 + (64 * c + 16 * k) * SW, HIDP * SW, 8 * SW, SW);
-          mma_bf16_warp(ty + ys * D, ad, bd, kIdY, (c > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ts_warp(ty + ys * D, tg + g * 32 + 8 * k, bd, kIdY, (c > 0 || k > 0) ? 1u : 0u);
         }
         mma_commit_warp(&bars[FB_A_EMPTY + g]);
       }
@@ -297,34 +315,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mma_commit_warp(&bars[FB_DONE]);
     mbar_drain(&bars[FB_DONE], 0);
-  } else if (warp >= 2 && warp <= 9) {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
-    const int g = (warp - 2) >> 2;          // warpgroup
+    const int e = (warp - kEpiWarp0) >> 2;  // warpgroup 0..3
+    const int pr = e >> 1;                  // pair: chunks c % 2 == pr, Y of tiles j % 2 == pr
+    const int hf = e & 1;                   // half of the chunk (32 hidden) / of the Y columns
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;          // token row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t abuf = smem_u32(smem + L::off_a + g * L::kA);
+    constexpr int kYHalf = D / 2;           // Y columns per warpgroup
     uint32_t j = 0, u = 0;
     TTT_TR_DECL
 
-    // Y epilogue of tile jj (head, tile), done by warpgroup jj % 2.
+    // Y epilogue of tile jj (head, tile): columns [hf*D/2, (hf+1)*D/2).
     auto y_epilogue = [&](uint32_t jj, int head, int tile) -> bool {
       const uint32_t ys = jj & 1;
       TTT_TR_LAP(0);
       if (!mbar_wait(&bars[FB_Y_FULL + ys], (jj >> 1) & 1, ab)) return false;
       TTT_TR_LAP(5);
       tc_fence_after();
-      float y[D];
-      const uint32_t yb = ty + ys * D + lane_off;
+      float y[kYHalf];
+      const uint32_t yb = ty + ys * D + hf * kYHalf + lane_off;
+      if (kYHalf >= 16) {
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        if (D >= 16 && c0 + 16 <= D) {
+        for (int c0 = 0; c0 < kYHalf; c0 += 16) {
           uint32_t r[16];
           tmem_ld16(yb + c0, r);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) y[c0 + i] = __uint_as_float(r[i]);
         }
+      } else {
+        uint32_t r[8];
+        tmem_ld8(yb, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(r[i]);
       }
       tc_fence_before();
       __syncwarp();
@@ -333,9 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars[FB_VP_FULL + ys], (jj >> 1) & 1, ab)) return false;
         const uint32_t vb = smem_u32(smem + L::off_vp + ys * L::kTile);
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
+        for (int ch = 0; ch < kYHalf / 8; ++ch) {
           uint32_t v0, v1, v2, v3;
-          ld_shared_v4(vb + swz(row * SW + ch * 16, SW), v0, v1, v2, v3);
+          ld_shared_v4(vb + swz(row * SW + (hf * kYHalf / 8 + ch) * 16, SW), v0, v1, v2, v3);
           y[8 * ch + 0] -= bf16lo(v0); y[8 * ch + 1] -= bf16hi(v0);
           y[8 * ch + 2] -= bf16lo(v1); y[8 * ch + 3] -= bf16hi(v1);
           y[8 * ch + 4] -= bf16lo(v2); y[8 * ch + 5] -= bf16hi(v2);
@@ -346,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const long long tok = static_cast<long long>(tile) * kTileM + row;
       if (tok < p.n) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + head) * D);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + head) * D + hf * kYHalf);
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
+        for (int ch = 0; ch < kYHalf / 8; ++ch) {
           uint4 v;
           v.x = pack_bf16x2(y[8 * ch + 0], y[8 * ch + 1]);
           v.y = pack_bf16x2(y[8 * ch + 2], y[8 * ch + 3]);
@@ -366,53 +392,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor cu;
     cu.init(it0, p.tiles);
     for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
-      for (int c = g; c < NC; c += 2, ++u) {
+      for (int c = pr; c < NC; c += 2, ++u) {
         TTT_TR_LAP(0);
-        if (!(ok = mbar_wait(&bars[FB_Z_FULL + g], u & 1, ab))) break;
+        if (!(ok = mbar_wait(&bars[FB_Z_FULL + pr], u & 1, ab))) break;
         TTT_TR_LAP(1);
         tc_fence_after();
-        uint32_t apk[32];  // 64 gate values of this row, bf16 pairs
-        const uint32_t zb = tz + g * 128 + lane_off;
+        // Z slot columns: [Z1 (32) | Z3 (32)] of hidden 64c + 0..31, then of 64c + 32..63;
+        // this warpgroup's half hf is columns 64*hf .. 64*hf + 63.
+        const uint32_t zb = tz + pr * 128 + hf * 64 + lane_off;
+        uint32_t gk[16];  // 32 gate values of this row as f16 pairs
 #pragma unroll
-        for (int sc = 0; sc < 2; ++sc) {
+        for (int part = 0; part < 2; ++part) {
+          uint32_t z1[16], z3[16];
+          tmem_ld16(zb + part * 16, z1);
+          tmem_ld16(zb + 32 + part * 16, z3);
+          tmem_wait_ld();
+          TTT_TR_LAP(7);
 #pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            uint32_t z1[16], z3[16];
-            tmem_ld16(zb + sc * 64 + qq * 16, z1);
-            tmem_ld16(zb + sc * 64 + 32 + qq * 16, z3);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              const float a0 = __uint_as_float(z1[i]), a1 = __uint_as_float(z1[i + 1]);
-              const float b0 = __uint_as_float(z3[i]), b1 = __uint_as_float(z3[i + 1]);
-              apk[(sc * 2 + qq) * 8 + i / 2] =
-                  pack_bf16x2(a0 * sigmoid_fast(a0) * b0, a1 * sigmoid_fast(a1) * b1);
-            }
-          }
+          for (int i = 0; i < 16; i += 2)
+            gk[part * 8 + i / 2] = gate_f16x2(__uint_as_float(z1[i]), __uint_as_float(z1[i + 1]),
+                                              __uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + g]);
+        if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + pr]);
         TTT_TR_LAP(2);
-        if (!(ok = mbar_wait(&bars[FB_A_EMPTY + g], (u & 1) ^ 1, ab))) break;
+        if (!(ok = mbar_wait(&bars[FB_A_EMPTY + pr], (u & 1) ^ 1, ab))) break;
         TTT_TR_LAP(3);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(abuf + swz(row * 128 + ch * 16, 128), apk[4 * ch], apk[4 * ch + 1], apk[4 * ch + 2],
-                       apk[4 * ch + 3]);
-        fence_proxy_async_smem();
+        tc_fence_after();
+        tmem_st16(tg + pr * 32 + hf * 16 + lane_off, gk);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[FB_A_FULL + g]);
+        if (lane == 0) mbar_arrive(&bars[FB_A_FULL + pr]);
         TTT_TR_LAP(4);
       }
       if (!ok) break;
-      if (j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) ok = y_epilogue(j - 1, prev_head, prev_tile);
+      if (j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(pr)) ok = y_epilogue(j - 1, prev_head, prev_tile);
       prev_head = cu.major;
       prev_tile = cu.tile;
     }
-    if (ok && j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(g)) y_epilogue(j - 1, prev_head, prev_tile);
+    if (ok && j >= 1 && ((j - 1) & 1) == static_cast<uint32_t>(pr)) y_epilogue(j - 1, prev_head, prev_tile);
     TTT_TR_LAP(0);
-    TTT_TR_DUMP(WRITE ? 0 : 1);
+    if (hf == 0 && pr == 0) TTT_TR_DUMP(WRITE ? 0 : 1);
   }
 
   tc_fence_before();

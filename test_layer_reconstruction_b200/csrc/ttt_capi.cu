@@ -58,19 +58,21 @@ int num_sms() {
 }
 
 struct Grids {
-  int fwd, bwd, max_contrib;
+  int fwd, bwd, bwd_groups, max_contrib;
 };
 
+// Forward: one CTA per SM over (head, tile) items.  Backward: groups of
+// `slices` CTAs over (head, tile) items, one hidden slice per CTA of a group.
 Grids grids_for(const Shape& s, int sms) {
   Grids g;
-  const long long fi = static_cast<long long>(s.H) * s.tiles;
-  const long long bi = static_cast<long long>(s.H) * s.slices * s.tiles;
-  g.fwd = static_cast<int>(std::min<long long>(sms, fi));
-  g.bwd = static_cast<int>(std::min<long long>(sms, bi));
+  const long long items = static_cast<long long>(s.H) * s.tiles;
+  g.fwd = static_cast<int>(std::min<long long>(sms, items));
+  g.bwd_groups = static_cast<int>(std::max<long long>(1, std::min<long long>(sms / s.slices, items)));
+  g.bwd = g.bwd_groups * s.slices;
   int mc = 1;
-  for (long long pair = 0; pair < static_cast<long long>(s.H) * s.slices; ++pair) {
-    const long long lo = owner_cta(pair * s.tiles, bi, g.bwd);
-    const long long hi = owner_cta(pair * s.tiles + s.tiles - 1, bi, g.bwd);
+  for (long long head = 0; head < s.H; ++head) {
+    const long long lo = owner_cta(head * s.tiles, items, g.bwd_groups);
+    const long long hi = owner_cta(head * s.tiles + s.tiles - 1, items, g.bwd_groups);
     mc = std::max<int>(mc, static_cast<int>(hi - lo + 1));
   }
   g.max_contrib = mc;
@@ -78,7 +80,7 @@ Grids grids_for(const Shape& s, int sms) {
 }
 
 struct Ws {
-  size_t status, w13, w2, vp, e, part, q, k, v, o, convw, th0, thout, total;
+  size_t status, w13, w2, w2h, vp, e, part, q, k, v, o, convw, th0, thout, total;
 };
 
 Ws ws_layout(const Shape& s, const Grids& g, int op) {
@@ -95,6 +97,7 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
   w.status = take(256);
   w.w13 = take(static_cast<size_t>(s.H) * 2 * s.hidp * s.D * 2);
   w.w2 = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
+  w.w2h = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
   if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST) {
     w.vp = take(tok_bytes);
     w.e = take(tok_bytes);
@@ -201,17 +204,20 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_EC
 int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float* w, uint16_t* out,
              cudaStream_t st) {
   ConvParams p;
-  p.V = reinterpret_cast<const uint4*>(V);
+  p.V = reinterpret_cast<const uint2*>(V);
   p.w = w;
-  p.out = reinterpret_cast<uint4*>(out);
+  p.out = reinterpret_cast<uint2*>(out);
   p.n_views = dm->n_views;
   p.gh = dm->grid_h;
   p.gw = dm->grid_w;
   p.n_special = dm->n_special;
   p.C = static_cast<int>(s.C);
-  const int g8 = p.C / 8;
-  const int block = std::min(128, (g8 + 31) / 32 * 32);
-  dim3 grid((g8 + block - 1) / block, dm->grid_h + 1, dm->n_views);
+  const int g4 = p.C / 4;
+  const int block = std::min(kConvThreads, (g4 + 31) / 32 * 32);
+  const long long items = static_cast<long long>(dm->n_views) * (dm->grid_h + 1);
+  const int sms = num_sms();
+  const long long persistent = static_cast<long long>(sms > 0 ? sms : 148) * 3;
+  dim3 grid(static_cast<unsigned>(std::min(items, persistent)), (g4 + block - 1) / block, 1);
   ProfScope prof(KK_CONV, st);
   shortconv_kernel<<<grid, block, 0, st>>>(p);
   return launch_status();
@@ -222,11 +228,12 @@ int run_pack(const Shape& s, const float* theta, const Ws& w, uint8_t* ws, cudaS
   p.theta = theta;
   p.w13_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w13);
   p.w2_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w2);
+  p.w2h_img = reinterpret_cast<__half*>(ws + w.w2h);
   p.heads = s.H;
   p.d = s.D;
   p.h = s.h;
   p.hidp = s.hidp;
-  const long long total = static_cast<long long>(s.H) * 3 * s.hidp * s.D;
+  const long long total = static_cast<long long>(s.H) * 4 * s.hidp * s.D;
   ProfScope prof(KK_PACK, st);
   pack_images_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(p);
   return launch_status();
@@ -269,7 +276,7 @@ int launch_bwd_t(const CUtensorMap& tk, const CUtensorMap& te, const BwdParams& 
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return TTT_ECUDA;
   ProfScope prof(KK_BWD, st);
-  k<<<grid, kThreads, smem, st>>>(tk, te, p);
+  k<<<grid, kBwdThreads, smem, st>>>(tk, te, p);
   return launch_status();
 }
 
@@ -324,7 +331,7 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   if (!make_token_map(&tk, K, s) || !make_token_map(&tvp, vp, s) || !make_token_map(&te, e, s)) return TTT_ECUDA;
   FwdParams fp;
   fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
-  fp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
+  fp.w2_img = reinterpret_cast<const __half*>(c.ws + c.w.w2h);
   fp.out = reinterpret_cast<__nv_bfloat16*>(e);
   fp.n = static_cast<int>(s.n);
   fp.heads = s.H;
@@ -332,7 +339,7 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   fp.status = status;
   BwdParams bp;
   bp.w13_img = fp.w13_img;
-  bp.w2_img = fp.w2_img;
+  bp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
   bp.partials = reinterpret_cast<float*>(c.ws + c.w.part);
   bp.n = fp.n;
   bp.heads = s.H;
@@ -349,8 +356,8 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   up.slices = s.slices;
   up.tiles = s.tiles;
   up.max_contrib = c.g.max_contrib;
-  up.n_items = static_cast<long long>(s.H) * s.slices * s.tiles;
-  up.grid = c.g.bwd;
+  up.n_items = static_cast<long long>(s.H) * s.tiles;
+  up.grid = c.g.bwd_groups;
   up.scale = lr * 2.0f / static_cast<float>(s.n);
   const long long red_threads = static_cast<long long>(s.H) * s.slices * 3 * 128 * s.D;
   for (int step = 0; step < steps; ++step) {
@@ -376,7 +383,7 @@ int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) 
   if (!make_token_map(&tq, Q, s)) return TTT_ECUDA;
   FwdParams fp;
   fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
-  fp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
+  fp.w2_img = reinterpret_cast<const __half*>(c.ws + c.w.w2h);
   fp.out = reinterpret_cast<__nv_bfloat16*>(O);
   fp.n = static_cast<int>(s.n);
   fp.heads = s.H;

@@ -1,7 +1,7 @@
 // update.cuh — the SGD step on the fast weights and the bf16 operand images.
 //
 // reduce_sgd: g = sum of the backward kernel's partials of a (head, hidden
-// slice) in CTA order (a fixed order, so the step is deterministic; Eq. 5 of
+// slice) in CTA-group order (a fixed order, so the step is deterministic; Eq. 5 of
 // VGG-T$^3$: Offline Feed-Forward 3D Reconstruction at Scale says the full
 // gradient is exactly the sum of the chunk gradients), then
 //   theta_out = theta_in - lr * (2/n) * g
@@ -14,7 +14,8 @@
 // swizzled by 8-row atoms), hidden units padded with zeros up to HIDP:
 //   W13 image, per head: for every 32-unit sub-chunk s, 32 rows of W1^T
 //     (hidden s*32+r) then 32 rows of W3^T;   2*HIDP rows.
-//   W2 image, per head: row j = W2[j][:];     HIDP rows.
+//   W2 image, per head: row j = W2[j][:];     HIDP rows (bf16, and again in
+//     f16 for the forward kernel, whose gate operand is f16).
 #pragma once
 #include "bwd.cuh"
 
@@ -25,8 +26,8 @@ struct UpdateParams {
   const float* theta_in;
   float* theta_out;
   int heads, d, h, slices, tiles, max_contrib;
-  long long n_items;   // heads * slices * tiles
-  int grid;            // CTAs of the backward kernel
+  long long n_items;   // heads * tiles
+  int grid;            // CTA groups of the backward kernel
   float scale;         // lr * 2 / n
 };
 
@@ -44,8 +45,9 @@ __global__ void reduce_sgd_kernel(const UpdateParams p) {
   const int head = static_cast<int>(pair / p.slices);
   const int hid = static_cast<int>(pair % p.slices) * 128 + hr;
   if (hid >= p.h) return;                                   // zero padding
-  const long long c_lo = owner_cta(pair * p.tiles, p.n_items, p.grid);
-  const long long c_hi = owner_cta(pair * p.tiles + p.tiles - 1, p.n_items, p.grid);
+  const long long first = static_cast<long long>(head) * p.tiles;
+  const long long c_lo = owner_cta(first, p.n_items, p.grid);
+  const long long c_hi = owner_cta(first + p.tiles - 1, p.n_items, p.grid);
   const float* src = p.partials + static_cast<size_t>(pair) * p.max_contrib * per_pair + e;
   float g = 0.f;
   for (long long c = 0; c <= c_hi - c_lo; ++c) g += src[c * per_pair];
@@ -61,6 +63,7 @@ struct PackParams {
   const float* theta;
   __nv_bfloat16* w13_img;
   __nv_bfloat16* w2_img;
+  __half* w2h_img;       // the W2 image again in f16 (B operand against the f16 gate)
   int heads, d, h, hidp;
 };
 
@@ -70,7 +73,7 @@ __global__ void pack_images_kernel(const PackParams p) {
   const long long n13 = static_cast<long long>(p.heads) * 2 * p.hidp * D;
   const long long n2 = static_cast<long long>(p.heads) * p.hidp * D;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n13 + n2) return;
+  if (idx >= n13 + 2 * n2) return;
   const size_t hdh = static_cast<size_t>(p.heads) * D * p.h;
   if (idx < n13) {
     const int col = static_cast<int>(idx % D);
@@ -88,7 +91,8 @@ __global__ void pack_images_kernel(const PackParams p) {
     *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w13_img + static_cast<size_t>(head) * 2 * p.hidp * D) + off) =
         __float2bfloat16_rn(v);
   } else {
-    const long long k = idx - n13;
+    const bool half = idx >= n13 + n2;
+    const long long k = idx - n13 - (half ? n2 : 0);
     const int col = static_cast<int>(k % D);
     const long long r_all = k / D;
     const int R = static_cast<int>(r_all % p.hidp);
@@ -96,8 +100,12 @@ __global__ void pack_images_kernel(const PackParams p) {
     float v = 0.f;
     if (R < p.h) v = p.theta[2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(R) * D + col];
     const uint32_t off = swz(static_cast<uint32_t>(R) * SW + col * 2, SW);
-    *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w2_img + static_cast<size_t>(head) * p.hidp * D) + off) =
-        __float2bfloat16_rn(v);
+    if (half)
+      *reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(p.w2h_img + static_cast<size_t>(head) * p.hidp * D) + off) =
+          __float2half_rn(v);
+    else
+      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w2_img + static_cast<size_t>(head) * p.hidp * D) +
+                                        off) = __float2bfloat16_rn(v);
   }
 }
 
