@@ -45,8 +45,8 @@ from typing import List, Sequence, Tuple
 import numpy as np
 
 __all__ = [
-    "Dims", "shortconv2d", "sigmoid", "swiglu_forward", "mse_loss", "mse_grad",
-    "sgd_write", "read", "layer", "LinearModel", "SwiGLUModel",
+    "Dims", "shortconv2d", "sigmoid", "swiglu_forward", "mse_loss", "mse_grad", "mse_grad_chunked",
+    "sgd_write", "read", "layer", "LinearModel", "SwiGLUModel", "ChunkedSwiGLUModel",
 ]
 
 
@@ -167,6 +167,38 @@ def mse_grad(K, Vp, W1, W3, W2) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     dZ1 = dA * Z3 * S * (1.0 + Z1 * (1.0 - S))
     dZ3 = dA * Z1 * S
     return K.T @ dZ1, K.T @ dZ3, dW2
+
+
+def mse_grad_chunked(K, Vp, W1, W3, W2, chunk: int):
+    """mse_grad summed over token chunks ([summary] Eq. 5: the gradient of the
+    total loss is the sum of the per-minibatch gradients), to bound memory on
+    long sequences.  Each chunk's gradient is normalised by its own length, so
+    it is weighted by len(chunk)/n."""
+    n = K.shape[0]
+    acc = [np.zeros_like(W1, dtype=np.float64), np.zeros_like(W3, dtype=np.float64),
+           np.zeros_like(W2, dtype=np.float64)]
+    for a in range(0, n, chunk):
+        b = min(n, a + chunk)
+        g = mse_grad(K[a:b], Vp[a:b], W1, W3, W2)
+        for p in range(3):
+            acc[p] += g[p] * ((b - a) / n)
+    return tuple(acc)
+
+
+class ChunkedSwiGLUModel:
+    """SwiGLU with the Eq. 5 chunked gradient (same values, bounded memory)."""
+
+    def __init__(self, chunk: int):
+        self.chunk = chunk
+
+    def forward(self, X, theta):
+        out = np.empty((X.shape[0], theta[2].shape[1]))
+        for a in range(0, X.shape[0], self.chunk):
+            out[a:a + self.chunk] = swiglu_forward(X[a:a + self.chunk], *theta)[0]
+        return out
+
+    def grad(self, X, Vp, theta):
+        return mse_grad_chunked(X, Vp, *theta, chunk=self.chunk)
 
 
 # ---------------------------------------------------------------------------

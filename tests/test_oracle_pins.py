@@ -256,6 +256,23 @@ def test_minibatch_gradient_decomposition_eq5():
         np.testing.assert_allclose(acc[p], full[p], rtol=1e-12, atol=1e-15)
 
 
+def test_chunked_gradient_equals_full_gradient():
+    """mse_grad_chunked (used on long sequences) restates Eq. 5: same values as mse_grad."""
+    n, d, h = 101, 4, 6
+    K = _unit_rows(rng.normal(size=(n, d))); Vp = rng.normal(size=(n, d))
+    th = _rand_theta(d, h, seed=17)
+    full = orc.mse_grad(K, Vp, *th)
+    for chunk in (1, 7, 50, 101, 500):
+        got = orc.mse_grad_chunked(K, Vp, *th, chunk=chunk)
+        for p in range(3):
+            np.testing.assert_allclose(got[p], full[p], rtol=1e-12, atol=1e-15)
+    m = orc.ChunkedSwiGLUModel(13)
+    a, _ = orc.sgd_write(K, Vp, th, 0.3, 2, model=m)
+    b, _ = orc.sgd_write(K, Vp, th, 0.3, 2)
+    for p in range(3):
+        np.testing.assert_allclose(a[p], b[p], rtol=1e-12, atol=1e-15)
+
+
 def test_fixed_point_zero_gradient():
     """If V' = T_theta0(K) the loss is 0, its gradient is 0 and theta stays put."""
     n, d, h = 30, 4, 8
