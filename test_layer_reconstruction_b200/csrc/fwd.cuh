@@ -367,8 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           y[8 * ch + 4] -= bf16lo(v2); y[8 * ch + 5] -= bf16hi(v2);
           y[8 * ch + 6] -= bf16lo(v3); y[8 * ch + 7] -= bf16hi(v3);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[FB_VP_EMPTY + ys]);
       }
       const long long tok = static_cast<long long>(tile) * kTileM + row;
       if (tok < p.n) {
@@ -382,6 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           v.w = pack_bf16x2(y[8 * ch + 6], y[8 * ch + 7]);
           dst[ch] = v;
         }
+      }
+      if (WRITE) {
+        // The V' stage is refilled by TMA (async proxy) once all eight warps
+        // have arrived.  An arrive right after the shared loads let the refill
+        // land before the last loads of some lanes had returned, so the stage
+        // is released only after the residual has been stored (the stores
+        // consume every loaded value), behind a generic-to-async proxy fence.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[FB_VP_EMPTY + ys]);
       }
       TTT_TR_LAP(6);
       return true;

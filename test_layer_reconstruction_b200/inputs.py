@@ -12,14 +12,21 @@ then the ``grid_h x grid_w`` patch grid in row-major order):
 * VGG-T^3 paper, Sec. 3.2 / App. A: per-head width 64 (VGGT width 1024 = 16 x 64),
   SwiGLU fast-weight MLP, 1 inner step for short collections and 2 at 1k views.
 
-Distributions: Q and K rows are L2-normalised N(0,1) draws per (token, head)
-row of length d (the pages' L2 normalisation of Q and K, Sec. 3.2), then
-rounded to bfloat16; V ~ N(0,1) rounded to bfloat16; depthwise 3x3 weights
-~ N(0, 1/9); fast weights Xavier-normal with std sqrt(2 / (d + h)).
+Distributions.  In the layer, Q, K and V are projections of the same token
+features, so V at a token is partly predictable from K at that token.  The
+draws keep that structure: every (token, head) row has one latent x ~ N(0, I_d),
+and with per-head projections P_Q, P_K, P_V ~ N(0, 1/d) (d x d, one draw per
+sequence)
+    K = x P_K / ||x P_K||,  Q = x P_Q / ||x P_Q||   (the pages' L2 normalisation
+                                                     of Q and K, Sec. 3.2)
+    V = x P_V                                       (rows of unit variance),
+each then rounded to bfloat16.  Depthwise 3x3 weights ~ N(0, 1/9); fast
+weights Xavier-normal with std sqrt(2 / (d + h)).
 
-Every view of every token tensor is drawn from its own generator, seeded by a
+Every view's latents are drawn from their own generator, seeded by a
 SplitMix64 mix of (seed, tensor id, view index), so any subset or permutation
-of views reproduces the same values.
+of views reproduces the same values.  Held-out views draw their latents from
+the held-out seed and share the sequence's projections.
 """
 from __future__ import annotations
 
@@ -37,7 +44,7 @@ __all__ = [
 _MASK64 = (1 << 64) - 1
 
 # tensor ids of the counter-based seeding
-_TID_K, _TID_Q, _TID_V, _TID_CONV, _TID_W1, _TID_W3, _TID_W2 = range(7)
+_TID_K, _TID_Q, _TID_V, _TID_CONV, _TID_W1, _TID_W3, _TID_W2, _TID_X = range(8)
 
 
 def _splitmix64(x: int) -> int:
@@ -130,14 +137,26 @@ def view_token_index(cfg: LayerConfig, view: int, y: int, x: int) -> int:
     return view * cfg.tokens_per_view + cfg.n_special + y * cfg.grid_w + x
 
 
-def _token_tensor(cfg, tensor_id, views, device, normalise, seed) -> torch.Tensor:
-    parts = []
-    for v in views:
-        r = _randn((cfg.tokens_per_view, cfg.heads, cfg.d), seed, tensor_id, v, device)
+def _latents(cfg, views, device, seed) -> torch.Tensor:
+    """One N(0, I_d) latent per (token, head) row, drawn view by view."""
+    parts = [_randn((cfg.tokens_per_view, cfg.heads, cfg.d), seed, _TID_X, v, device) for v in views]
+    return torch.cat(parts, 0) if parts else torch.zeros(0, cfg.heads, cfg.d, device=device)
+
+
+def _projection(cfg, tensor_id, device) -> torch.Tensor:
+    """Per-head d x d projection ~ N(0, 1/d), drawn from the sequence seed."""
+    return _randn((cfg.heads, cfg.d, cfg.d), cfg.seed, tensor_id, 0, device) * (1.0 / math.sqrt(cfg.d))
+
+
+def _project(X, P, normalise) -> torch.Tensor:
+    out = torch.empty_like(X)
+    step = 1 << 16   # bounded temporaries on long sequences
+    for a in range(0, X.shape[0], step):
+        r = torch.einsum("thd,hde->the", X[a:a + step], P)
         if normalise:
             r = r / torch.linalg.vector_norm(r, dim=-1, keepdim=True)
-        parts.append(r)
-    return torch.cat(parts, 0) if parts else torch.zeros(0, cfg.heads, cfg.d, device=device)
+        out[a:a + step] = r
+    return out
 
 
 def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] = None,
@@ -155,11 +174,13 @@ def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] =
     seed = cfg.heldout_seed if heldout else cfg.seed
     out: Dict[str, torch.Tensor] = {}
     rnd = (lambda t: t) if cfg.fp32_inputs else bf16_round
-    out["Q"] = rnd(_token_tensor(cfg, _TID_Q, views, device, True, seed))
+    X = _latents(cfg, views, device, seed)
+    out["Q"] = rnd(_project(X, _projection(cfg, _TID_Q, device), True))
     if heldout:
         return out
-    out["K"] = rnd(_token_tensor(cfg, _TID_K, views, device, True, seed))
-    out["V"] = rnd(_token_tensor(cfg, _TID_V, views, device, False, seed))
+    out["K"] = rnd(_project(X, _projection(cfg, _TID_K, device), True))
+    out["V"] = rnd(_project(X, _projection(cfg, _TID_V, device), False))
+    del X
     C = cfg.heads * cfg.d
     out["conv_w"] = _randn((C, 3, 3), seed, _TID_CONV, 0, device) * (1.0 / 3.0)
     std = math.sqrt(2.0 / (cfg.d + cfg.h))
