@@ -178,8 +178,10 @@ def _kernel_work(cfg):
         "swiglu_fwd_residual": ("tensor", 6.0 * d * h * n * H),      # Z1, Z3, Y
         "swiglu_bwd_partials": ("tensor", 8.0 * d * h * n * H),      # dA, dW1, dW3, dW2
         "swiglu_fwd_read": ("tensor", 6.0 * d * h * n * H),
-        "pack_theta": ("hbm", 3 * H * d * h * 4 + 3 * H * 128 * math.ceil(h / 128) * d * 2),
-        "reduce_sgd": ("hbm", 0),
+        # read theta (f32); write the W1|W3 bf16 image and the bf16 and f16 W2 images
+        "pack_theta": ("hbm", 3 * H * d * h * 4 + 4 * H * 128 * math.ceil(h / 128) * d * 2),
+        # read theta, write theta* (the split-K partials it also reads are a by-product of the tiling)
+        "reduce_sgd": ("hbm", 2 * 3 * H * d * h * 4),
     }
 
 
@@ -278,7 +280,7 @@ def run_ours(args, cfg):
                          "frac": achieved / peak if peak else None}
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches_per_step"])
     dk = kernels[dom]
-    traffic = _traffic_from_profiles(dom)
+    traffic = _traffic_from_profiles(dom, cfg.name)
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                 "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic,
                 "peak_source": f"{peaks['source']} ({'sustained bf16' if dk['bound'] == 'tensor' else 'HBM copy'})"}
@@ -337,15 +339,32 @@ def run_ours(args, cfg):
     return 0
 
 
-def _traffic_from_profiles(kernel: str):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary, when one matches the current build."""
+def _kernel_source_digest() -> str:
+    """sha256 over the CUDA sources (csrc/*.cu, csrc/*.cuh, by name)."""
+    import hashlib
+    d = os.path.join(ROOT, "test_layer_reconstruction_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def _traffic_from_profiles(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/traffic.json), or None when the counters were taken on other
+    kernel sources or another workload."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         with open(path) as f:
             t = json.load(f)
-        return t.get(kernel)
+        if t.get("source_sha256") != _kernel_source_digest() or t.get("workload") != workload:
+            return None
+        return t["bytes_per_launch"].get(kernel)
     except Exception:
         return None
 
