@@ -5,39 +5,57 @@
 // Feed-Forward 3D Reconstruction at Scale, Sec. 3.4, Eq. 3; the gradient is a
 // sum of per-token terms, Eq. 5) with residual E = T(K) - V' from the forward
 // kernel, the chain rule through T(x) = (silu(x W1) * (x W3)) W2 gives, per
-// token tile (G = (2/n) E; the 2/n is applied in the update):
+// token (G = (2/n) E; the 2/n is applied in the update):
 //   Z1 = K W1, Z3 = K W3, S = sigmoid(Z1)                      (recomputed)
 //   dA = E W2^T
 //   dZ1 = dA * Z3 * S * (1 + Z1 (1 - S)),  dZ3 = dA * Z1 * S,  A = Z1 S Z3
 //   dW1^T += dZ1^T K,  dW3^T += dZ3^T K,  dW2 += A^T E
-// CTA work = (head, 128-wide slice of the hidden units, contiguous range of
-// 128-token tiles); the CTAs of one group share the tile range, one slice
-// each.  dW for the slice stays in TMEM for the whole range and is written
-// once per (head, slice) segment to a partial buffer.  The update kernel sums
-// the partials of a (head, slice) in group order, so the result is
-// deterministic.
 //
-// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + sub-chunk MMA
-// issuer, warp 10 dW MMA issuer, warps 2-9 two epilogue warpgroups.  Per tile the
-// slice is walked in 4 sub-chunks of 32 hidden units, each with
-//   Z  = K * [W1 | W3]_sub   (M=128 tokens, N=64, K=d)
-//   dA = E * W2_sub^T        (M=128 tokens, N=32, K=d)
-// in one of 3 TMEM slots; the epilogue writes A, dZ1, dZ3 (bf16) to shared
-// memory and the dW MMAs (M=128 hidden, N=d, K=128 tokens, both operands
-// MN-major) of a tile go out as soon as that is done.
+// Hidden-major formulation.  All products are taken with the hidden units on
+// the 128 TMEM lanes:
+//   U^T = (W1/2)^T K^T, Z3^T = W3^T K^T     (M=128 hidden, N=48 tokens, K=d;
+//        A = the slice's W1^T/2 and W3^T rows kept in TMEM, B = the K tile)
+//   dA^T = W2 E^T                           (same shape; A = the slice's W2
+//        rows in shared memory, B = the E tile)
+// The epilogue thread of hidden unit r evaluates the chain rule for 16 tokens
+// and writes 2*dZ1^T, dZ3^T and A^T back to TMEM as packed bf16, over the Z
+// columns it has just read; that is exactly the A operand layout of
+//   dW1^T += (2 dZ1^T) K, dW3^T += dZ3^T K, dW2 += A^T E   (M=128 hidden, N=d,
+//        K=16 tokens; B = the same K/E tile, read MN-major)
+// (the factor 2 is removed in the update), so no intermediate goes through
+// shared memory.  With u = z1/2 and t = tanh(u): sigmoid(z1) = (1+t)/2,
+// silu(z1) = u (1+t) and 2 d silu/dz1 = (1+t) + u (1 - t^2).
+//
+// CTA work = (head, 128-wide slice of the hidden units, contiguous range of
+// 48-token units); the CTAs of one group share the unit range, one slice
+// each.  dW of the slice stays in TMEM for the whole range and is written once
+// per (head, slice) segment to a partial buffer; the update kernel sums the
+// partials of a (head, slice) in group order, so the result is deterministic.
+//
+// Warp roles: warp 0 TMA producer; warp 1 TMEM allocator and U/Z3/dA issuer;
+// warp 2 dW issuer; warp 3 idle; warps 4-15 three epilogue warpgroups, group g
+// owning tokens 16g..16g+15 of every unit.  The U/Z3 columns are double
+// buffered by unit parity, dA^T is single buffered (the epilogue empties it as
+// soon as the unit is ready).  Both issuers run warp-uniform loops with
+// precomputed descriptors and issue from one elected lane.
 #pragma once
 #include "fwd.cuh"
 
 namespace ttt {
 
-constexpr int kBwdThreads = 352;    // 11 warps: 0 producer, 1 sub-chunk issuer, 2-9 epilogue, 10 dW issuer
-constexpr int kBwdDwWarp = 10;
+constexpr int kUnit = 48;             // tokens per backward unit (N of the U/Z3/dA products)
+constexpr int kBwdThreads = 512;      // 16 warps
+constexpr int kBwdZWarp = 1;
+constexpr int kBwdDwWarp = 2;
+constexpr int kBwdEpiWarp0 = 4;
+constexpr int kBwdStages = 6;         // K/E ring depth
 
 struct BwdParams {
-  const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
-  const __nv_bfloat16* w2_img;   // per head: HIDP rows of D bf16 (sw-swizzled)
+  // Per head, per hidden row r < HIDP: [W1^T row / 2 | W3^T row | W2 row], D
+  // bf16 each (zero for r >= h); read as pairs (element 2c in the low half).
+  const uint32_t* wt_img;
   float* partials;               // [head*slices+slice][max_contrib][3][128][D] f32
-  int n, heads, tiles, slices;   // slices = HIDP / 128
+  int n, heads, units, slices;   // units = ceil(n / kUnit); slices = HIDP / 128
   int max_contrib;
   unsigned int* status;
 };
@@ -45,29 +63,31 @@ struct BwdParams {
 template <int D>
 struct BwdLayout {
   static constexpr int SW = 2 * D;
-  static constexpr uint32_t kW13 = 2u * 128 * D * 2;  // rows of one 128-wide slice
-  static constexpr uint32_t kW2 = 1u * 128 * D * 2;
-  static constexpr uint32_t kTile = 1u * kTileM * D * 2;
-  static constexpr uint32_t kBuf = 2u * kTileM * 64 * 2;  // [128 tok][128 hid] as 2 atoms of 64
-  static constexpr uint32_t off_w13 = 0;
-  static constexpr uint32_t off_w2 = off_w13 + kW13;
-  static constexpr uint32_t off_k = off_w2 + kW2;
-  static constexpr uint32_t off_e = off_k + 2 * kTile;
-  static constexpr uint32_t off_a = off_e + 2 * kTile;
-  static constexpr uint32_t off_dz1 = off_a + kBuf;
-  static constexpr uint32_t off_dz3 = off_dz1 + kBuf;
-  static constexpr uint32_t off_bar = off_dz3 + kBuf;
-  static constexpr int kNumBars = 24;
+  static constexpr uint32_t kBox = 1u * kUnit * D * 2;                  // bytes of one TMA box
+  static constexpr uint32_t kStage = (kBox + 1023u) / 1024u * 1024u;    // swizzle-period aligned
+  static constexpr uint32_t kW2 = 128u * D * 2;                         // the slice's W2 rows (K-major)
+  static constexpr uint32_t off_w2 = 0;
+  static constexpr uint32_t off_k = off_w2 + (kW2 + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t off_e = off_k + kBwdStages * kStage;
+  static constexpr uint32_t off_bar = off_e + kBwdStages * kStage;
+  static constexpr int kNumBars = 32;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
-  static_assert(off_k % 1024 == 0 && off_e % 1024 == 0 && off_a % 1024 == 0, "1 KiB alignment");
+  // TMEM columns
+  static constexpr uint32_t cW = 0;                 // W1^T/2, W3^T rows: D/2 columns each
+  static constexpr uint32_t cDW = D;                // dW1^T (x2), dW3^T, dW2: D columns each
+  static constexpr uint32_t cZ = cDW + 3 * D;       // 2 buffers of [U^T | Z3^T], 2*kUnit columns each
+  static constexpr uint32_t cDA = cZ + 4 * kUnit;   // dA^T, kUnit columns
+  static_assert(cDA + kUnit <= 512, "tensor memory");
 };
 
 enum BwdBar {
-  BB_W_FULL = 0, BB_W_EMPTY = 1, BB_KE_FULL = 2, BB_KE_EMPTY = 4, BB_SL_FULL = 6, BB_SL_EMPTY = 9,
-  BB_DZ_FULL = 12, BB_DZ_EMPTY = 13, BB_ACC_FULL = 14, BB_ACC_EMPTY = 15, BB_DONE = 16
+  BB_KE_FULL = 0, BB_KE_EMPTY = kBwdStages, BB_W_FULL = 2 * kBwdStages, BB_W_EMPTY, BB_U_FULL,
+  BB_Z_EMPTY = BB_U_FULL + 2, BB_DA_EMPTY = BB_Z_EMPTY + 2, BB_P_FULL, BB_ACC_FULL = BB_P_FULL + 6, BB_ACC_EMPTY,
+  BB_DONE
 };
+static_assert(BB_DONE < 32, "barrier count");
 
-// Group (of CTAs) that owns flattened (head, tile) item i under the static
+// Group (of CTAs) that owns flattened (head, unit) item i under the static
 // partition [floor(g*N/G), floor((g+1)*N/G)).
 __host__ __device__ inline long long owner_cta(long long i, long long n_items, long long grid) {
   return ((i + 1) * grid - 1) / n_items;
@@ -79,8 +99,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int SW = L::SW;
-  constexpr uint32_t kSlot = 96;       // TMEM columns per sub-chunk slot
-  constexpr uint32_t kDw = 288;        // first dW column
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
@@ -90,35 +108,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // CTAs come in groups of `slices`: CTA group*slices + s handles hidden slice s
-  // of the group's (head, tile) range, so the CTAs of a group read the same K/E
+  // of the group's (head, unit) range, so the CTAs of a group read the same K/E
   // tiles at about the same time and all but the first find them in L2.
   const int slice_id = blockIdx.x % p.slices;
   const int group = blockIdx.x / p.slices;
   const int groups = gridDim.x / p.slices;
-  const long long total = static_cast<long long>(p.heads) * p.tiles;
+  const long long total = static_cast<long long>(p.heads) * p.units;
   const long long it0 = total * group / groups;
   const long long it1 = total * (group + 1) / groups;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(&bars[BB_W_FULL], 1);
-    mbar_init(&bars[BB_W_EMPTY], 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(&bars[BB_KE_FULL + s], 1);
       mbar_init(&bars[BB_KE_EMPTY + s], 1);
     }
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(&bars[BB_SL_FULL + s], 1);
-      mbar_init(&bars[BB_SL_EMPTY + s], 4);
+    mbar_init(&bars[BB_W_FULL], 12);     // every epilogue warp writes part of the weights
+    mbar_init(&bars[BB_W_EMPTY], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[BB_U_FULL + b], 1);
+      mbar_init(&bars[BB_Z_EMPTY + b], 1);
     }
-    mbar_init(&bars[BB_DZ_FULL], 8);
-    mbar_init(&bars[BB_DZ_EMPTY], 1);
+    mbar_init(&bars[BB_DA_EMPTY], 12);
+    // per (buffer, token group): a warpgroup can refill buffer b only after the
+    // dW MMAs of the unit before have drained it, so no phase is ever skipped
+    for (int i = 0; i < 6; ++i) mbar_init(&bars[BB_P_FULL + i], 4);
     mbar_init(&bars[BB_ACC_FULL], 1);
-    mbar_init(&bars[BB_ACC_EMPTY], 8);
+    mbar_init(&bars[BB_ACC_EMPTY], 12);
     mbar_init(&bars[BB_DONE], 2);
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kBwdZWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -133,96 +153,79 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       TTT_TR_DECL
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_e);
-      long long cur_pair = -1;
-      int head = 0, slice = 0;
-      uint32_t wl = 0, j = 0;
-      Cursor pf;
-      pf.init(it0, p.tiles);
-      for (int k = 0; k < kPrefetchAhead && pf.it < it1; ++k, pf.next(p.tiles)) {
-        tma_prefetch_l2_2d(&tm_k, pf.major * D, pf.tile * kTileM);
-        tma_prefetch_l2_2d(&tm_e, pf.major * D, pf.tile * kTileM);
-      }
       Cursor cu;
-      cu.init(it0, p.tiles);
-      for (; cu.it < it1; cu.next(p.tiles), ++j) {
-        const int pair = cu.major * p.slices + slice_id;
-        const int tile = cu.tile;
-        if (pair != cur_pair) {
-          head = cu.major;
-          slice = slice_id;
-          TTT_TR_LAP(0);
-          if (wl > 0 && !mbar_wait(&bars[BB_W_EMPTY], (wl - 1) & 1, ab)) break;
-          TTT_TR_LAP(2);
-          mbar_arrive_expect_tx(&bars[BB_W_FULL], L::kW13 + L::kW2);
-          const size_t hidp = static_cast<size_t>(p.slices) * 128;
-          const __nv_bfloat16* w13 = p.w13_img + (static_cast<size_t>(head) * 2 * hidp + slice * 256) * D;
-          const __nv_bfloat16* w2 = p.w2_img + (static_cast<size_t>(head) * hidp + slice * 128) * D;
-          bulk_load_pieces(smem + L::off_w13, w13, L::kW13, &bars[BB_W_FULL]);
-          bulk_load_pieces(smem + L::off_w2, w2, L::kW2, &bars[BB_W_FULL]);
-          ++wl;
-          cur_pair = pair;
-        }
-        const int s = j & 1;
-        if (pf.it < it1) {
-          tma_prefetch_l2_2d(&tm_k, pf.major * D, pf.tile * kTileM);
-          tma_prefetch_l2_2d(&tm_e, pf.major * D, pf.tile * kTileM);
-          pf.next(p.tiles);
-        }
+      cu.init(it0, p.units);
+      uint32_t s = 0, ph = 0, issued = 0;
+      for (; cu.it < it1; cu.next(p.units), ++issued) {
         TTT_TR_LAP(0);
-        if (!mbar_wait(&bars[BB_KE_EMPTY + s], ((j >> 1) & 1) ^ 1, ab)) break;
+        if (!mbar_wait(&bars[BB_KE_EMPTY + s], ph ^ 1, ab)) break;
         TTT_TR_LAP(1);
-        mbar_arrive_expect_tx(&bars[BB_KE_FULL + s], 2 * L::kTile);
-        tma_load_2d(smem + L::off_k + s * L::kTile, &tm_k, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
-        tma_load_2d(smem + L::off_e + s * L::kTile, &tm_e, &bars[BB_KE_FULL + s], head * D, tile * kTileM);
+        mbar_arrive_expect_tx(&bars[BB_KE_FULL + s], 2 * L::kBox);
+        tma_load_2d(smem + L::off_k + s * L::kStage, &tm_k, &bars[BB_KE_FULL + s], cu.major * D, cu.tile * kUnit);
+        tma_load_2d(smem + L::off_e + s * L::kStage, &tm_e, &bars[BB_KE_FULL + s], cu.major * D, cu.tile * kUnit);
+        if (++s == kBwdStages) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       TTT_TR_LAP(0);
       TTT_TR_DUMP(2);
-      if (wl > 0) mbar_drain(&bars[BB_W_FULL], (wl - 1) & 1);
-      for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) mbar_drain(&bars[BB_KE_FULL + (jj & 1)], (jj >> 1) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ sub-chunk issuer
-    // Z = K * [W1 | W3]_sub and dA = E * W2_sub^T into one of 3 TMEM slots.
-    constexpr uint32_t kIdZ = idesc_bf16(128, 64, false, false);
-    constexpr uint32_t kIdDA = idesc_bf16(128, 32, false, false);
-    const uint32_t w13 = smem_u32(smem + L::off_w13);
-    const uint32_t w2 = smem_u32(smem + L::off_w2);
-    TTT_TR_DECL
-    Cursor sc;
-    sc.init(it0, p.tiles);
-    int cur_pair = -1;
-    uint32_t sj = 0, kc = 0, wl = 0;
-    bool ok = true;
-    for (; sc.it < it1 && ok; sc.next(p.tiles), ++sj) {
-      if (sc.major != cur_pair) {
-        if (cur_pair >= 0) mma_commit_warp(&bars[BB_W_EMPTY]);
-        if (!(ok = mbar_wait_warp(&bars[BB_W_FULL], wl & 1, ab))) break;
-        ++wl;
-        cur_pair = sc.major;
+      // Drain: the last load issued into each stage has landed before exit.
+      const uint32_t last = issued < static_cast<uint32_t>(kBwdStages) ? issued : kBwdStages;
+      for (uint32_t b = 0; b < last; ++b) {
+        const uint32_t jj = issued - 1 - b;
+        mbar_drain(&bars[BB_KE_FULL + jj % kBwdStages], (jj / kBwdStages) & 1);
       }
-      const int s = sj & 1;
-      TTT_TR_LAP(0);
-      if (!(ok = mbar_wait_warp(&bars[BB_KE_FULL + s], (sj >> 1) & 1, ab))) break;
-      TTT_TR_LAP(1);
-      const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
-      const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
-      for (int ssc = 0; ssc < 4; ++ssc, ++kc) {
-        const uint32_t slot = kc % 3, use = kc / 3;
+    }
+  } else if (warp == kBwdZWarp) {
+    // ------------------------------------------------------------ U / Z3 / dA issuer
+    constexpr uint32_t kId = idesc_bf16(128, kUnit, false, false);
+    const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
+    const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
+    const uint64_t dw2 = smem_desc(smem_u32(smem + L::off_w2), 0, 8 * SW, SW);
+    const uint32_t tW = tbase + L::cW, tDA = tbase + L::cDA;
+    TTT_TR_DECL
+    Cursor zc;
+    zc.init(it0, p.units);
+    int cur_head = -1;
+    uint32_t s = 0, ph = 0, j = 0, seg = 0;
+    bool ok = true;
+    for (; zc.it < it1 && ok; zc.next(p.units), ++j) {
+      if (zc.major != cur_head) {
+        if (seg > 0) mma_commit_warp(&bars[BB_W_EMPTY]);
         TTT_TR_LAP(0);
-        if (!(ok = mbar_wait_warp(&bars[BB_SL_EMPTY + slot], (use & 1) ^ 1, ab))) break;
-        TTT_TR_LAP(2);
-        tc_fence_after();
-        const uint32_t tsl = tbase + slot * kSlot;
+        if (!(ok = mbar_wait_warp(&bars[BB_W_FULL], seg & 1, ab))) break;
+        TTT_TR_LAP(4);
+        ++seg;
+        cur_head = zc.major;
+      }
+      const uint32_t b = j & 1;
+      TTT_TR_LAP(0);
+      if (!(ok = mbar_wait_warp(&bars[BB_KE_FULL + s], ph, ab))) break;
+      TTT_TR_LAP(1);
+      const uint64_t soff = (s * L::kStage) >> 4;
+      const uint64_t dk = dk0 + soff, de = de0 + soff;
+      // dA^T of this unit once the epilogue has read the previous one.
+      if (!(ok = mbar_wait_warp(&bars[BB_DA_EMPTY], (j & 1) ^ 1, ab))) break;
+      TTT_TR_LAP(2);
+      tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_bf16_warp(tsl, smem_desc(ks + 32 * k, 0, 8 * SW, SW),
-                        smem_desc(w13 + 64 * ssc * SW + 32 * k, 0, 8 * SW, SW), kIdZ, k > 0 ? 1u : 0u);
+      for (int k = 0; k < D / 16; ++k) mma_bf16_warp(tDA, dw2 + 2 * k, de + 2 * k, kId, k > 0 ? 1u : 0u);
+      // U^T, Z3^T into buffer b once the dW MMAs of unit j-2 have read it.
+      if (!(ok = mbar_wait_warp(&bars[BB_Z_EMPTY + b], ((j >> 1) & 1) ^ 1, ab))) break;
+      TTT_TR_LAP(5);
+      tc_fence_after();
+      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_bf16_warp(tsl + 64, smem_desc(es + 32 * k, 0, 8 * SW, SW),
-                        smem_desc(w2 + 32 * ssc * SW + 32 * k, 0, 8 * SW, SW), kIdDA, k > 0 ? 1u : 0u);
-        mma_commit_warp(&bars[BB_SL_FULL + slot]);
-        TTT_TR_LAP(3);
+      for (int k = 0; k < D / 16; ++k) mma_bf16_ts_warp(tz, tW + 8 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        mma_bf16_ts_warp(tz + kUnit, tW + D / 2 + 8 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
+      mma_commit_warp(&bars[BB_U_FULL + b]);
+      TTT_TR_LAP(3);
+      if (++s == kBwdStages) {
+        s = 0;
+        ph ^= 1;
       }
     }
     TTT_TR_DUMP(2);
@@ -230,74 +233,85 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_drain(&bars[BB_DONE], 0);
   } else if (warp == kBwdDwWarp) {
     // ------------------------------------------------------------ dW issuer
-    // dW1^T += dZ1^T K, dW3^T += dZ3^T K, dW2 += A^T E once the epilogue has
-    // written A, dZ1, dZ3 of the tile.  This warp's commit releases the K/E
-    // stage: the tile's sub-chunk MMAs completed before the epilogue could
-    // write its dZ, so every reader of the stage is done.
-    constexpr uint32_t kIdW = idesc_bf16(128, D, true, true);
-    const uint32_t sa = smem_u32(smem + L::off_a);
-    const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
-    const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
+    // dW1^T += (2 dZ1^T) K, dW3^T += dZ3^T K, dW2 += A^T E per 16-token group
+    // as soon as its epilogue warpgroup has written it.  The unit's last
+    // commits release its U/Z3 buffer and its K/E stage: the unit's other
+    // MMAs completed before the epilogue could read their results, so every
+    // reader of the stage is done.
+    constexpr uint32_t kIdW = idesc_bf16(128, D, false, true);
+    const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
+    const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
+    const uint32_t tDW = tbase + L::cDW;
+    TTT_TR_DECL
     Cursor wc;
-    wc.init(it0, p.tiles);
-    uint32_t wj = 0, wseg = 0;
+    wc.init(it0, p.units);
+    uint32_t s = 0, j = 0, seg = 0;
     bool ok = true;
-    for (; wc.it < it1 && ok; wc.next(p.tiles), ++wj) {
+    for (; wc.it < it1 && ok; wc.next(p.units), ++j) {
       const bool first = (wc.it == it0) || wc.tile == 0;
-      const bool last = (wc.it == it1 - 1) || wc.tile == p.tiles - 1;
-      if (!(ok = mbar_wait_warp(&bars[BB_DZ_FULL], wj & 1, ab))) break;
-      if (first && wseg > 0 && !(ok = mbar_wait_warp(&bars[BB_ACC_EMPTY], (wseg - 1) & 1, ab))) break;
-      tc_fence_after();
-      const int s = wj & 1;
-      const uint32_t ks = smem_u32(smem + L::off_k + s * L::kTile);
-      const uint32_t es = smem_u32(smem + L::off_e + s * L::kTile);
-#pragma unroll
-      for (int k = 0; k < kTileM / 16; ++k) {
-        const uint32_t acc = (first && k == 0) ? 0u : 1u;
-        const uint64_t bk = smem_desc(ks + k * 16 * SW, 0, 8 * SW, SW);
-        const uint64_t be = smem_desc(es + k * 16 * SW, 0, 8 * SW, SW);
-        mma_bf16_warp(tbase + kDw, smem_desc(sdz1 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
-        mma_bf16_warp(tbase + kDw + D, smem_desc(sdz3 + k * 2048, 16384, 1024, 128), bk, kIdW, acc);
-        mma_bf16_warp(tbase + kDw + 2 * D, smem_desc(sa + k * 2048, 16384, 1024, 128), be, kIdW, acc);
+      const bool last = (wc.it == it1 - 1) || wc.tile == p.units - 1;
+      if (first && seg > 0) {
+        TTT_TR_LAP(0);
+        if (!(ok = mbar_wait_warp(&bars[BB_ACC_EMPTY], (seg - 1) & 1, ab))) break;
+        TTT_TR_LAP(4);
       }
-      mma_commit_warp(&bars[BB_DZ_EMPTY]);
+      const uint32_t b = j & 1;
+      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit);
+      const uint64_t soff = (s * L::kStage) >> 4;
+      const uint64_t dk = dk0 + soff, de = de0 + soff;
+#pragma unroll
+      for (int g = 0; g < 3; ++g) {
+        TTT_TR_LAP(0);
+        if (!(ok = mbar_wait_warp(&bars[BB_P_FULL + 3 * b + g], (j >> 1) & 1, ab))) break;
+        TTT_TR_LAP(1);
+        tc_fence_after();
+        const uint32_t acc = (first && g == 0) ? 0u : 1u;
+        const uint64_t go = (16u * g * SW) >> 4;
+        mma_bf16_ts_warp(tDW, tz + 16 * g, dk + go, kIdW, acc);
+        mma_bf16_ts_warp(tDW + D, tz + 16 * g + 8, dk + go, kIdW, acc);
+        mma_bf16_ts_warp(tDW + 2 * D, tz + kUnit + 16 * g, de + go, kIdW, acc);
+        TTT_TR_LAP(2);
+      }
+      if (!ok) break;
+      mma_commit_warp(&bars[BB_Z_EMPTY + b]);
       mma_commit_warp(&bars[BB_KE_EMPTY + s]);
       if (last) {
         mma_commit_warp(&bars[BB_ACC_FULL]);   // segment done: the epilogue dumps dW
-        ++wseg;
+        ++seg;
       }
+      if (++s == kBwdStages) s = 0;
     }
+    TTT_TR_DUMP(2);
     mma_commit_warp(&bars[BB_DONE]);
     mbar_drain(&bars[BB_DONE], 0);
-  } else if (warp >= 2 && warp <= 9) {
+  } else if (warp >= kBwdEpiWarp0) {
     // ------------------------------------------------------------ epilogue
-    const int g = (warp - 2) >> 2;
-    const int q = warp & 3;
-    const int row = q * 32 + lane;            // token row (sub-chunks), hidden row (dW dump)
+    const int g = (warp - kBwdEpiWarp0) >> 2;  // token group of every unit; weight / dW matrix it moves
+    const int q = warp & 3;                    // TMEM lane quadrant
+    const int row = q * 32 + lane;             // hidden unit within the slice
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t sa = smem_u32(smem + L::off_a);
-    const uint32_t sdz1 = smem_u32(smem + L::off_dz1);
-    const uint32_t sdz3 = smem_u32(smem + L::off_dz3);
-    uint32_t j = 0, seg = 0;
+    uint32_t j = 0, seg = 0, dumps = 0;
     long long cur_pair = -1;
     bool ok = true;
     TTT_TR_DECL
 
-    // Write dW of the finished segment (pair) to its partial slot.
+    // Write dW of the finished segment (pair) to its partial slot: warpgroup g
+    // moves matrix g (2 dW1^T, dW3^T, dW2), row = hidden unit.
     auto dump = [&](long long pair) -> bool {
       TTT_TR_LAP(0);
-      if (!mbar_wait(&bars[BB_ACC_FULL], seg & 1, ab)) return false;
+      if (!mbar_wait(&bars[BB_ACC_FULL], dumps & 1, ab)) return false;
       TTT_TR_LAP(5);
       tc_fence_after();
-      const long long first_item = (pair / p.slices) * static_cast<long long>(p.tiles);
+      const long long first_item = (pair / p.slices) * static_cast<long long>(p.units);
       const long long contrib = group - owner_cta(first_item, total, groups);
-      float* dst = p.partials + (static_cast<size_t>(pair) * p.max_contrib + contrib) * (3u * 128u * D);
-      for (int grp = g; grp < 3 * D / 16; grp += 2) {
+      float* dst = p.partials + (static_cast<size_t>(pair) * p.max_contrib + contrib) * (3u * 128u * D) +
+                   (static_cast<size_t>(g) * 128 + row) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t r[16];
-        tmem_ld16(tbase + kDw + grp * 16 + lane_off, r);
+        tmem_ld16(tbase + L::cDW + g * D + c0 + lane_off, r);
         tmem_wait_ld();
-        const int m = grp * 16 / D, col = grp * 16 % D;
-        float4* o = reinterpret_cast<float4*>(dst + (static_cast<size_t>(m) * 128 + row) * D + col);
+        float4* o = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           o[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
@@ -306,88 +320,110 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[BB_ACC_EMPTY]);
-      ++seg;
+      ++dumps;
       TTT_TR_LAP(6);
       return true;
     };
 
+    // Weights of a (head, slice): warpgroup 0 writes W1^T/2 rows and warpgroup
+    // 1 W3^T rows into TMEM, warpgroup 2 the W2 rows into shared memory (the
+    // K-major, swizzled A operand of dA^T).
+    auto load_weights = [&](int head) -> bool {
+      if (seg > 0 && !mbar_wait(&bars[BB_W_EMPTY], (seg - 1) & 1, ab)) return false;
+      tc_fence_after();
+      const size_t hidp = static_cast<size_t>(p.slices) * 128;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          p.wt_img + ((static_cast<size_t>(head) * hidp + slice_id * 128 + row) * 3 + g) * (D / 2));
+      if (g == 2) {
+        const uint32_t base = smem_u32(smem + L::off_w2);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 x = __ldg(src + c);
+          st_shared_v4(base + swz(static_cast<uint32_t>(row) * SW + c * 16, SW), x.x, x.y, x.z, x.w);
+        }
+        fence_proxy_async_smem();
+      } else if constexpr (D >= 32) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          uint32_t w[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = __ldg(src + c0 / 4 + v);
+            w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+          }
+          tmem_st16(tbase + L::cW + g * (D / 2) + c0 + lane_off, w);
+        }
+        tmem_wait_st();
+      } else {
+        uint32_t w[8];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const uint4 x = __ldg(src + v);
+          w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+        }
+        tmem_st8(tbase + L::cW + g * (D / 2) + lane_off, w);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BB_W_FULL]);
+      ++seg;
+      return true;
+    };
+
     Cursor cu;
-    cu.init(it0, p.tiles);
-    for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
+    cu.init(it0, p.units);
+    for (; cu.it < it1 && ok; cu.next(p.units), ++j) {
       const long long pair = static_cast<long long>(cu.major) * p.slices + slice_id;
       if (pair != cur_pair) {
         if (cur_pair >= 0 && !(ok = dump(cur_pair))) break;
+        if (!(ok = load_weights(cu.major))) break;
         cur_pair = pair;
       }
-      bool waited_buf = false;
-      for (int sc = g; sc < 4; sc += 2) {
-        const uint32_t kc = j * 4 + sc;
-        const uint32_t slot = kc % 3, use = kc / 3;
-        TTT_TR_LAP(0);
-        if (!(ok = mbar_wait(&bars[BB_SL_FULL + slot], use & 1, ab))) break;
-        TTT_TR_LAP(1);
-        tc_fence_after();
-        const uint32_t tsl = tbase + slot * kSlot + lane_off;
-        // Load the whole sub-chunk (Z1, Z3, dA), return the slot to the MMA
-        // issuer at once, then compute from registers.
-        uint32_t zz1[2][16], zz3[2][16], zda[2][16];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld16(tsl + half * 16, zz1[half]);
-          tmem_ld16(tsl + 32 + half * 16, zz3[half]);
-          tmem_ld16(tsl + 64 + half * 16, zda[half]);
-        }
-        tmem_wait_ld();
-        TTT_TR_LAP(7);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[BB_SL_EMPTY + slot]);
-        uint32_t pa[16], pz1[16], pz3[16];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t (&z1)[16] = zz1[half];
-          const uint32_t (&z3)[16] = zz3[half];
-          const uint32_t (&da)[16] = zda[half];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            // Packed bf16 arithmetic on two hidden units (the outputs are the
-            // bf16 operands of the dW MMAs): with s = sigmoid(z1) =
-            // (1 + tanh(z1/2))/2, silu = z1 s, A = silu z3, and
-            // d silu/dz1 = s (1 + z1 (1 - s)):
-            //   dZ1 = dA * (z3 s + z3 s * z1 (1 - s)),  dZ3 = dA * silu.
-            const uint32_t b1 = pack_bf16x2(__uint_as_float(z1[i]), __uint_as_float(z1[i + 1]));
-            const uint32_t b3 = pack_bf16x2(__uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
-            const uint32_t bd = pack_bf16x2(__uint_as_float(da[i]), __uint_as_float(da[i + 1]));
-            const uint32_t sg = bfma2(btanh2(bmul2(b1, kBf2Half)), kBf2Half, kBf2Half);
-            const uint32_t silu = bmul2(b1, sg);
-            const uint32_t tt = bmul2(b3, sg);
-            const uint32_t w = bmul2(b1, bfma2(sg, kBf2NegOne, kBf2One));
-            pa[half * 8 + i / 2] = bmul2(silu, b3);
-            pz1[half * 8 + i / 2] = bmul2(bd, bfma2(tt, w, tt));
-            pz3[half * 8 + i / 2] = bmul2(bd, silu);
-          }
-        }
-        TTT_TR_LAP(2);
-        if (!waited_buf) {
-          if (!(ok = mbar_wait(&bars[BB_DZ_EMPTY], (j & 1) ^ 1, ab))) break;
-          waited_buf = true;
-        }
-        TTT_TR_LAP(3);
-        // hidden unit (within the slice) sc*32 + 8v + e  ->  atom sc/2, 16-byte chunk (sc%2)*4 + v
-        const uint32_t base = (sc >> 1) * 16384u;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint32_t off = base + swz(row * 128 + ((sc & 1) * 4 + v) * 16, 128);
-          st_shared_v4(sa + off, pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
-          st_shared_v4(sdz1 + off, pz1[4 * v], pz1[4 * v + 1], pz1[4 * v + 2], pz1[4 * v + 3]);
-          st_shared_v4(sdz3 + off, pz3[4 * v], pz3[4 * v + 1], pz3[4 * v + 2], pz3[4 * v + 3]);
-        }
-      }
-      if (!ok) break;
-      fence_proxy_async_smem();
+      const uint32_t b = j & 1;
+      TTT_TR_LAP(0);
+      if (!(ok = mbar_wait(&bars[BB_U_FULL + b], (j >> 1) & 1, ab))) break;
+      TTT_TR_LAP(1);
+      tc_fence_after();
+      uint32_t zu[16], z3[16], da[16];
+      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit) + 16 * g + lane_off;
+      tmem_ld16(tz, zu);
+      tmem_ld16(tz + kUnit, z3);
+      tmem_ld16(tbase + L::cDA + 16 * g + lane_off, da);
+      tmem_wait_ld();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[BB_DZ_FULL]);
-      TTT_TR_LAP(4);
+      if (lane == 0) mbar_arrive(&bars[BB_DA_EMPTY]);
+      TTT_TR_LAP(2);
+      uint32_t pz1[8], pz3[8], pa[8];
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        // Packed bf16 arithmetic on two tokens of this hidden unit (the outputs
+        // are the bf16 A operands of the dW MMAs), with u = z1/2, t = tanh(u):
+        //   silu = u (1+t),  2 dsilu/dz1 = (1+t) + u (1 - t^2),
+        //   2 dZ1 = dA z3 (2 dsilu/dz1),  dZ3 = dA silu,  A = silu z3.
+        const uint32_t bu = pack_bf16x2(__uint_as_float(zu[i]), __uint_as_float(zu[i + 1]));
+        const uint32_t b3 = pack_bf16x2(__uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
+        const uint32_t bd = pack_bf16x2(__uint_as_float(da[i]), __uint_as_float(da[i + 1]));
+        const uint32_t t = btanh2(bu);
+        const uint32_t s2 = bfma2(t, kBf2One, kBf2One);                 // 1 + t
+        const uint32_t silu = bmul2(bu, s2);
+        const uint32_t om = bfma2(t ^ 0x80008000u, t, kBf2One);          // 1 - t^2
+        const uint32_t q2 = bfma2(bu, om, s2);                          // 2 dsilu/dz1
+        pz1[i / 2] = bmul2(bmul2(bd, b3), q2);
+        pz3[i / 2] = bmul2(bd, silu);
+        pa[i / 2] = bmul2(silu, b3);
+      }
+      TTT_TR_LAP(3);
+      // Over the U/Z3 columns of this warpgroup's tokens, already read above.
+      tmem_st8(tz, pz1);
+      tmem_st8(tz + 8, pz3);
+      tmem_st8(tz + kUnit, pa);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BB_P_FULL + 3 * b + g]);
+      TTT_TR_LAP(7);
     }
     if (ok && cur_pair >= 0) dump(cur_pair);
     TTT_TR_LAP(0);
@@ -396,7 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kBwdZWarp) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }

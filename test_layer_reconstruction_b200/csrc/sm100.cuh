@@ -242,6 +242,11 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // 32 lanes x 32 bits, 16 consecutive columns per thread, registers -> TMEM.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -302,7 +307,7 @@ __host__ __device__ constexpr uint32_t swz(uint32_t off, int sw) {
 // the host reads them with ttt_trace_read.  Off by default: the macros expand
 // to nothing.
 #ifdef TTT_TRACE
-constexpr int kTraceKernels = 3, kTraceWarps = 11, kTraceSlots = 8;
+constexpr int kTraceKernels = 3, kTraceWarps = 20, kTraceSlots = 8;
 // Defined here: the library is a single translation unit.
 __device__ unsigned long long g_ttt_trace[kTraceKernels * kTraceWarps * kTraceSlots];
 struct Tracer {
@@ -319,7 +324,7 @@ struct Tracer {
     t = now;
   }
   __device__ __forceinline__ void dump(int kernel, int warp, int lane) {
-    if (lane != 0) return;
+    if (lane != 0 || warp >= kTraceWarps) return;
     for (int i = 0; i < kTraceSlots; ++i)
       atomicAdd(&g_ttt_trace[(kernel * kTraceWarps + warp) * kTraceSlots + i], acc[i]);
   }

@@ -24,7 +24,7 @@ size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
 struct Shape {
   long long n;   // tokens
-  int H, D, h, hidp, tiles, slices;
+  int H, D, h, hidp, tiles, slices, units;
   long long C;   // H * D channels
 };
 
@@ -46,6 +46,7 @@ int check_dims(const ttt_dims* dm, Shape* s) {
   s->hidp = (dm->h + 127) / 128 * 128;
   s->slices = s->hidp / 128;
   s->tiles = static_cast<int>((n + kTileM - 1) / kTileM);
+  s->units = static_cast<int>((n + kUnit - 1) / kUnit);
   s->C = static_cast<long long>(dm->heads) * dm->d;
   return TTT_OK;
 }
@@ -61,18 +62,20 @@ struct Grids {
   int fwd, bwd, bwd_groups, max_contrib;
 };
 
-// Forward: one CTA per SM over (head, tile) items.  Backward: groups of
-// `slices` CTAs over (head, tile) items, one hidden slice per CTA of a group.
+// Forward: one CTA per SM over (head, 128-token tile) items.  Backward: groups
+// of `slices` CTAs over (head, 48-token unit) items, one hidden slice per CTA
+// of a group.
 Grids grids_for(const Shape& s, int sms) {
   Grids g;
   const long long items = static_cast<long long>(s.H) * s.tiles;
   g.fwd = static_cast<int>(std::min<long long>(sms, items));
-  g.bwd_groups = static_cast<int>(std::max<long long>(1, std::min<long long>(sms / s.slices, items)));
+  const long long units = static_cast<long long>(s.H) * s.units;
+  g.bwd_groups = static_cast<int>(std::max<long long>(1, std::min<long long>(sms / s.slices, units)));
   g.bwd = g.bwd_groups * s.slices;
   int mc = 1;
   for (long long head = 0; head < s.H; ++head) {
-    const long long lo = owner_cta(head * s.tiles, items, g.bwd_groups);
-    const long long hi = owner_cta(head * s.tiles + s.tiles - 1, items, g.bwd_groups);
+    const long long lo = owner_cta(head * s.units, units, g.bwd_groups);
+    const long long hi = owner_cta(head * s.units + s.units - 1, units, g.bwd_groups);
     mc = std::max<int>(mc, static_cast<int>(hi - lo + 1));
   }
   g.max_contrib = mc;
@@ -80,7 +83,7 @@ Grids grids_for(const Shape& s, int sms) {
 }
 
 struct Ws {
-  size_t status, w13, w2, w2h, vp, e, part, q, k, v, o, convw, th0, thout, total;
+  size_t status, w13, w2h, wt, vp, e, part, q, k, v, o, convw, th0, thout, total;
 };
 
 Ws ws_layout(const Shape& s, const Grids& g, int op) {
@@ -96,9 +99,9 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
   const size_t theta_bytes = 3ull * s.H * s.D * s.h * 4;
   w.status = take(256);
   w.w13 = take(static_cast<size_t>(s.H) * 2 * s.hidp * s.D * 2);
-  w.w2 = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
   w.w2h = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
   if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST) {
+    w.wt = take(static_cast<size_t>(s.H) * s.hidp * 3 * s.D * 2);
     w.vp = take(tok_bytes);
     w.e = take(tok_bytes);
     w.part = take(static_cast<size_t>(s.H) * s.slices * g.max_contrib * 3ull * 128 * s.D * 4);
@@ -133,14 +136,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D view [n rows][C bf16] of a token tensor; box = D columns x 128 rows,
+// 2-D view [n rows][C bf16] of a token tensor; box = D columns x `rows` rows,
 // swizzled by rows of 2*D bytes (the layout the kernels' descriptors expect).
-bool make_token_map(CUtensorMap* m, const void* base, const Shape& s) {
+bool make_token_map(CUtensorMap* m, const void* base, const Shape& s, int rows = kTileM) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(s.C), static_cast<cuuint64_t>(s.n)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(s.C) * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(s.D), static_cast<cuuint32_t>(kTileM)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(s.D), static_cast<cuuint32_t>(rows)};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle sw = s.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                           : (s.D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -223,17 +226,18 @@ int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float*
   return launch_status();
 }
 
-int run_pack(const Shape& s, const float* theta, const Ws& w, uint8_t* ws, cudaStream_t st) {
+// Operand images of theta; the backward kernel's weight rows only when `with_wt`.
+int run_pack(const Shape& s, const float* theta, const Ws& w, uint8_t* ws, bool with_wt, cudaStream_t st) {
   PackParams p;
   p.theta = theta;
   p.w13_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w13);
-  p.w2_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w2);
   p.w2h_img = reinterpret_cast<__half*>(ws + w.w2h);
+  p.wt_img = with_wt ? reinterpret_cast<__nv_bfloat16*>(ws + w.wt) : nullptr;
   p.heads = s.H;
   p.d = s.D;
   p.h = s.h;
   p.hidp = s.hidp;
-  const long long total = static_cast<long long>(s.H) * 4 * s.hidp * s.D;
+  const long long total = static_cast<long long>(s.H) * (with_wt ? 6 : 3) * s.hidp * s.D;
   ProfScope prof(KK_PACK, st);
   pack_images_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(p);
   return launch_status();
@@ -327,8 +331,10 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
       return TTT_ECUDA;
     return TTT_OK;
   }
-  CUtensorMap tk, tvp, te;
-  if (!make_token_map(&tk, K, s) || !make_token_map(&tvp, vp, s) || !make_token_map(&te, e, s)) return TTT_ECUDA;
+  CUtensorMap tk, tvp, tku, teu;
+  if (!make_token_map(&tk, K, s) || !make_token_map(&tvp, vp, s) || !make_token_map(&tku, K, s, kUnit) ||
+      !make_token_map(&teu, e, s, kUnit))
+    return TTT_ECUDA;
   FwdParams fp;
   fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
   fp.w2_img = reinterpret_cast<const __half*>(c.ws + c.w.w2h);
@@ -338,12 +344,11 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   fp.tiles = s.tiles;
   fp.status = status;
   BwdParams bp;
-  bp.w13_img = fp.w13_img;
-  bp.w2_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w2);
+  bp.wt_img = reinterpret_cast<const uint32_t*>(c.ws + c.w.wt);
   bp.partials = reinterpret_cast<float*>(c.ws + c.w.part);
   bp.n = fp.n;
   bp.heads = s.H;
-  bp.tiles = s.tiles;
+  bp.units = s.units;
   bp.slices = s.slices;
   bp.max_contrib = c.g.max_contrib;
   bp.status = status;
@@ -354,17 +359,17 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   up.d = s.D;
   up.h = s.h;
   up.slices = s.slices;
-  up.tiles = s.tiles;
+  up.units = s.units;
   up.max_contrib = c.g.max_contrib;
-  up.n_items = static_cast<long long>(s.H) * s.tiles;
+  up.n_items = static_cast<long long>(s.H) * s.units;
   up.grid = c.g.bwd_groups;
   up.scale = lr * 2.0f / static_cast<float>(s.n);
   const long long red_threads = static_cast<long long>(s.H) * s.slices * 3 * 128 * s.D;
   for (int step = 0; step < steps; ++step) {
     const float* th_in = step == 0 ? theta0 : theta_out;
-    if ((rc = run_pack(s, th_in, c.w, c.ws, c.st)) != TTT_OK) return rc;
+    if ((rc = run_pack(s, th_in, c.w, c.ws, true, c.st)) != TTT_OK) return rc;
     if ((rc = launch_fwd<true>(s, tk, tvp, fp, c.g.fwd, c.st)) != TTT_OK) return rc;
-    if ((rc = launch_bwd(s, tk, te, bp, c.g.bwd, c.st)) != TTT_OK) return rc;
+    if ((rc = launch_bwd(s, tku, teu, bp, c.g.bwd, c.st)) != TTT_OK) return rc;
     up.theta_in = th_in;
     {
       ProfScope prof(KK_REDUCE, c.st);
@@ -377,7 +382,7 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
 
 int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
   const Shape& s = c.s;
-  int rc = run_pack(s, theta, c.w, c.ws, c.st);
+  int rc = run_pack(s, theta, c.w, c.ws, false, c.st);
   if (rc != TTT_OK) return rc;
   CUtensorMap tq;
   if (!make_token_map(&tq, Q, s)) return TTT_ECUDA;

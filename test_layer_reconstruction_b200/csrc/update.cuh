@@ -9,13 +9,16 @@
 // here).  theta_out may alias theta_in: each element is read and written by
 // one thread.
 //
-// pack_images: theta (f32) -> bf16 round-to-nearest-even operand images laid
-// out exactly as the kernels' shared-memory tiles (rows of D elements,
-// swizzled by 8-row atoms), hidden units padded with zeros up to HIDP:
-//   W13 image, per head: for every 32-unit sub-chunk s, 32 rows of W1^T
-//     (hidden s*32+r) then 32 rows of W3^T;   2*HIDP rows.
-//   W2 image, per head: row j = W2[j][:];     HIDP rows (bf16, and again in
-//     f16 for the forward kernel, whose gate operand is f16).
+// pack_images: theta (f32) -> round-to-nearest-even operand images, hidden
+// units padded with zeros up to HIDP:
+//   W13 image (bf16), per head, laid out as the forward kernel's shared-memory
+//     tile (rows of D elements, swizzled by 8-row atoms): for every 32-unit
+//     sub-chunk s, 32 rows of W1^T (hidden s*32+r) then 32 rows of W3^T.
+//   W2 image (f16, same tiling), per head: row j = W2[j][:]; the forward
+//     kernel's gate operand is f16.
+//   WT image (bf16, plain rows; write path only), per head and hidden unit r:
+//     [W1^T row r / 2 | W3^T row r | W2 row r], the backward kernel's weight
+//     rows (halving is exact in bf16).
 #pragma once
 #include "bwd.cuh"
 
@@ -25,8 +28,8 @@ struct UpdateParams {
   const float* partials;
   const float* theta_in;
   float* theta_out;
-  int heads, d, h, slices, tiles, max_contrib;
-  long long n_items;   // heads * tiles
+  int heads, d, h, slices, units, max_contrib;
+  long long n_items;   // heads * units
   int grid;            // CTA groups of the backward kernel
   float scale;         // lr * 2 / n
 };
@@ -45,9 +48,9 @@ __global__ void reduce_sgd_kernel(const UpdateParams p) {
   const int head = static_cast<int>(pair / p.slices);
   const int hid = static_cast<int>(pair % p.slices) * 128 + hr;
   if (hid >= p.h) return;                                   // zero padding
-  const long long first = static_cast<long long>(head) * p.tiles;
+  const long long first = static_cast<long long>(head) * p.units;
   const long long c_lo = owner_cta(first, p.n_items, p.grid);
-  const long long c_hi = owner_cta(first + p.tiles - 1, p.n_items, p.grid);
+  const long long c_hi = owner_cta(first + p.units - 1, p.n_items, p.grid);
   const float* src = p.partials + static_cast<size_t>(pair) * p.max_contrib * per_pair + e;
   float g = 0.f;
   for (long long c = 0; c <= c_hi - c_lo; ++c) g += src[c * per_pair];
@@ -56,14 +59,15 @@ __global__ void reduce_sgd_kernel(const UpdateParams p) {
   if (m == 0) off = static_cast<size_t>(head) * D * p.h + static_cast<size_t>(i) * p.h + hid;
   else if (m == 1) off = hdh + static_cast<size_t>(head) * D * p.h + static_cast<size_t>(i) * p.h + hid;
   else off = 2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(hid) * D + i;
-  p.theta_out[off] = p.theta_in[off] - p.scale * g;
+  // the backward kernel accumulates 2 dW1^T (its chain rule runs on z1/2): halve it, exactly
+  p.theta_out[off] = p.theta_in[off] - (m == 0 ? 0.5f * p.scale : p.scale) * g;
 }
 
 struct PackParams {
   const float* theta;
   __nv_bfloat16* w13_img;
-  __nv_bfloat16* w2_img;
-  __half* w2h_img;       // the W2 image again in f16 (B operand against the f16 gate)
+  __half* w2h_img;
+  __nv_bfloat16* wt_img;  // null: not written
   int heads, d, h, hidp;
 };
 
@@ -72,8 +76,9 @@ __global__ void pack_images_kernel(const PackParams p) {
   const int D = p.d, SW = 2 * D;
   const long long n13 = static_cast<long long>(p.heads) * 2 * p.hidp * D;
   const long long n2 = static_cast<long long>(p.heads) * p.hidp * D;
+  const long long nt = p.wt_img ? 3 * n2 : 0;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n13 + 2 * n2) return;
+  if (idx >= n13 + n2 + nt) return;
   const size_t hdh = static_cast<size_t>(p.heads) * D * p.h;
   if (idx < n13) {
     const int col = static_cast<int>(idx % D);
@@ -90,9 +95,8 @@ __global__ void pack_images_kernel(const PackParams p) {
     const uint32_t off = swz(static_cast<uint32_t>(R) * SW + col * 2, SW);
     *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w13_img + static_cast<size_t>(head) * 2 * p.hidp * D) + off) =
         __float2bfloat16_rn(v);
-  } else {
-    const bool half = idx >= n13 + n2;
-    const long long k = idx - n13 - (half ? n2 : 0);
+  } else if (idx < n13 + n2) {
+    const long long k = idx - n13;
     const int col = static_cast<int>(k % D);
     const long long r_all = k / D;
     const int R = static_cast<int>(r_all % p.hidp);
@@ -100,12 +104,26 @@ __global__ void pack_images_kernel(const PackParams p) {
     float v = 0.f;
     if (R < p.h) v = p.theta[2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(R) * D + col];
     const uint32_t off = swz(static_cast<uint32_t>(R) * SW + col * 2, SW);
-    if (half)
-      *reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(p.w2h_img + static_cast<size_t>(head) * p.hidp * D) + off) =
-          __float2half_rn(v);
-    else
-      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w2_img + static_cast<size_t>(head) * p.hidp * D) +
-                                        off) = __float2bfloat16_rn(v);
+    *reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(p.w2h_img + static_cast<size_t>(head) * p.hidp * D) + off) =
+        __float2half_rn(v);
+  } else {
+    // WT: element idx = ((head * HIDP + r) * 3 + m) * D + col
+    const long long k = idx - n13 - n2;
+    const int col = static_cast<int>(k % D);
+    const int m = static_cast<int>((k / D) % 3);
+    const long long hr = k / (3LL * D);
+    const int r = static_cast<int>(hr % p.hidp);
+    const int head = static_cast<int>(hr / p.hidp);
+    float v = 0.f;
+    if (r < p.h) {
+      if (m < 2) {
+        v = p.theta[m * hdh + static_cast<size_t>(head) * D * p.h + static_cast<size_t>(col) * p.h + r];
+        if (m == 0) v *= 0.5f;   // W1^T / 2: the backward kernel's products give z1/2 directly
+      } else {
+        v = p.theta[2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(r) * D + col];
+      }
+    }
+    p.wt_img[k] = __float2bfloat16_rn(v);
   }
 }
 
