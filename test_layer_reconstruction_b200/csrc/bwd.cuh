@@ -12,19 +12,24 @@
 //   dW1^T += dZ1^T K,  dW3^T += dZ3^T K,  dW2 += A^T E
 //
 // Hidden-major formulation.  All products are taken with the hidden units on
-// the 128 TMEM lanes:
-//   U^T = (W1/2)^T K^T, Z3^T = W3^T K^T     (M=128 hidden, N=48 tokens, K=d;
-//        A = the slice's W1^T/2 and W3^T rows kept in TMEM, B = the K tile)
-//   dA^T = W2 E^T                           (same shape; A = the slice's W2
-//        rows in shared memory, B = the E tile)
+// the 128 TMEM lanes (M=128 hidden, N=48 tokens, K=d):
+//   U^T = (W1/2)^T K^T   A = the slice's W1^T/2 rows kept in TMEM (TS)
+//   Z3^T = W3^T K^T      A = the slice's W3^T rows in shared memory (SS)
+//   dA^T = W2 E^T        A = the slice's W2 rows in shared memory (SS)
 // The epilogue thread of hidden unit r evaluates the chain rule for 16 tokens
-// and writes 2*dZ1^T, dZ3^T and A^T back to TMEM as packed bf16, over the Z
-// columns it has just read; that is exactly the A operand layout of
+// and writes 2*dZ1^T, dZ3^T and A^T back to TMEM as packed bf16 (2 dZ1^T and
+// dZ3^T over the U columns it has just read, A^T into a small ring); that is
+// exactly the A operand layout of
 //   dW1^T += (2 dZ1^T) K, dW3^T += dZ3^T K, dW2 += A^T E   (M=128 hidden, N=d,
 //        K=16 tokens; B = the same K/E tile, read MN-major)
 // (the factor 2 is removed in the update), so no intermediate goes through
 // shared memory.  With u = z1/2 and t = tanh(u): sigmoid(z1) = (1+t)/2,
 // silu(z1) = u (1+t) and 2 d silu/dz1 = (1+t) + u (1 - t^2).
+//
+// Buffering (TMEM, 512 columns at d=64): U is triple buffered and is the only
+// buffer whose reuse waits for the dW MMAs, so a unit's epilogue never waits
+// on the dW products of the unit before; Z3^T and dA^T are single buffered
+// (the epilogue empties them as soon as a unit is ready); A^T has two slots.
 //
 // CTA work = (head, 128-wide slice of the hidden units, contiguous range of
 // 48-token units); the CTAs of one group share the unit range, one slice
@@ -34,10 +39,8 @@
 //
 // Warp roles: warp 0 TMA producer; warp 1 TMEM allocator and U/Z3/dA issuer;
 // warp 2 dW issuer; warp 3 idle; warps 4-15 three epilogue warpgroups, group g
-// owning tokens 16g..16g+15 of every unit.  The U/Z3 columns are double
-// buffered by unit parity, dA^T is single buffered (the epilogue empties it as
-// soon as the unit is ready).  Both issuers run warp-uniform loops with
-// precomputed descriptors and issue from one elected lane.
+// owning tokens 16g..16g+15 of every unit.  Both issuers run warp-uniform loops
+// with precomputed descriptors and issue from one elected lane.
 #pragma once
 #include "fwd.cuh"
 
@@ -49,6 +52,8 @@ constexpr int kBwdZWarp = 1;
 constexpr int kBwdDwWarp = 2;
 constexpr int kBwdEpiWarp0 = 4;
 constexpr int kBwdStages = 6;         // K/E ring depth
+constexpr int kBwdUBufs = 3;          // U^T buffers
+constexpr int kBwdPaSlots = 2;        // A^T slots
 
 struct BwdParams {
   // Per head, per hidden row r < HIDP: [W1^T row / 2 | W3^T row | W2 row], D
@@ -65,27 +70,30 @@ struct BwdLayout {
   static constexpr int SW = 2 * D;
   static constexpr uint32_t kBox = 1u * kUnit * D * 2;                  // bytes of one TMA box
   static constexpr uint32_t kStage = (kBox + 1023u) / 1024u * 1024u;    // swizzle-period aligned
-  static constexpr uint32_t kW2 = 128u * D * 2;                         // the slice's W2 rows (K-major)
-  static constexpr uint32_t off_w2 = 0;
-  static constexpr uint32_t off_k = off_w2 + (kW2 + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t kWRows = (128u * D * 2 + 1023u) / 1024u * 1024u;  // 128 weight rows (K-major)
+  static constexpr uint32_t off_w3 = 0;
+  static constexpr uint32_t off_w2 = off_w3 + kWRows;
+  static constexpr uint32_t off_k = off_w2 + kWRows;
   static constexpr uint32_t off_e = off_k + kBwdStages * kStage;
   static constexpr uint32_t off_bar = off_e + kBwdStages * kStage;
-  static constexpr int kNumBars = 32;
+  static constexpr int kNumBars = 40;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
   // TMEM columns
-  static constexpr uint32_t cW = 0;                 // W1^T/2, W3^T rows: D/2 columns each
-  static constexpr uint32_t cDW = D;                // dW1^T (x2), dW3^T, dW2: D columns each
-  static constexpr uint32_t cZ = cDW + 3 * D;       // 2 buffers of [U^T | Z3^T], 2*kUnit columns each
-  static constexpr uint32_t cDA = cZ + 4 * kUnit;   // dA^T, kUnit columns
-  static_assert(cDA + kUnit <= 512, "tensor memory");
+  static constexpr uint32_t cW1 = 0;                          // W1^T/2 rows: D/2 columns
+  static constexpr uint32_t cDW = (D / 2 + 15) / 16 * 16;     // 2 dW1^T, dW3^T, dW2: D columns each
+  static constexpr uint32_t cU = cDW + 3 * D;                 // kBwdUBufs x kUnit
+  static constexpr uint32_t cZ3 = cU + kBwdUBufs * kUnit;     // kUnit
+  static constexpr uint32_t cDA = cZ3 + kUnit;                // kUnit
+  static constexpr uint32_t cPA = cDA + kUnit;                // kBwdPaSlots x 3 groups x 8
+  static_assert(cPA + kBwdPaSlots * 24 <= 512, "tensor memory");
 };
 
 enum BwdBar {
-  BB_KE_FULL = 0, BB_KE_EMPTY = kBwdStages, BB_W_FULL = 2 * kBwdStages, BB_W_EMPTY, BB_U_FULL,
-  BB_Z_EMPTY = BB_U_FULL + 2, BB_DA_EMPTY = BB_Z_EMPTY + 2, BB_P_FULL, BB_ACC_FULL = BB_P_FULL + 6, BB_ACC_EMPTY,
-  BB_DONE
+  BB_KE_FULL = 0, BB_KE_EMPTY = kBwdStages, BB_W_FULL = 2 * kBwdStages, BB_W_EMPTY, BB_FULL,
+  BB_U_EMPTY = BB_FULL + kBwdUBufs, BB_ZD_EMPTY = BB_U_EMPTY + kBwdUBufs, BB_P_FULL,
+  BB_PA_EMPTY = BB_P_FULL + 3 * kBwdUBufs, BB_ACC_FULL = BB_PA_EMPTY + kBwdPaSlots, BB_ACC_EMPTY, BB_DONE
 };
-static_assert(BB_DONE < 32, "barrier count");
+static_assert(BB_DONE < 40, "barrier count");
 
 // Group (of CTAs) that owns flattened (head, unit) item i under the static
 // partition [floor(g*N/G), floor((g+1)*N/G)).
@@ -125,14 +133,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&bars[BB_W_FULL], 12);     // every epilogue warp writes part of the weights
     mbar_init(&bars[BB_W_EMPTY], 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars[BB_U_FULL + b], 1);
-      mbar_init(&bars[BB_Z_EMPTY + b], 1);
+    for (int b = 0; b < kBwdUBufs; ++b) {
+      mbar_init(&bars[BB_FULL + b], 1);
+      mbar_init(&bars[BB_U_EMPTY + b], 1);
     }
-    mbar_init(&bars[BB_DA_EMPTY], 12);
-    // per (buffer, token group): a warpgroup can refill buffer b only after the
-    // dW MMAs of the unit before have drained it, so no phase is ever skipped
-    for (int i = 0; i < 6; ++i) mbar_init(&bars[BB_P_FULL + i], 4);
+    mbar_init(&bars[BB_ZD_EMPTY], 12);
+    // per (U buffer, token group): a warpgroup reuses buffer b only after the
+    // dW MMAs of the unit that last used it have drained it, so no phase is
+    // ever skipped
+    for (int i = 0; i < 3 * kBwdUBufs; ++i) mbar_init(&bars[BB_P_FULL + i], 4);
+    for (int i = 0; i < kBwdPaSlots; ++i) mbar_init(&bars[BB_PA_EMPTY + i], 1);
     mbar_init(&bars[BB_ACC_FULL], 1);
     mbar_init(&bars[BB_ACC_EMPTY], 12);
     mbar_init(&bars[BB_DONE], 2);
@@ -182,13 +192,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr uint32_t kId = idesc_bf16(128, kUnit, false, false);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
     const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
+    const uint64_t dw3 = smem_desc(smem_u32(smem + L::off_w3), 0, 8 * SW, SW);
     const uint64_t dw2 = smem_desc(smem_u32(smem + L::off_w2), 0, 8 * SW, SW);
-    const uint32_t tW = tbase + L::cW, tDA = tbase + L::cDA;
+    const uint32_t tW1 = tbase + L::cW1, tZ3 = tbase + L::cZ3, tDA = tbase + L::cDA;
     TTT_TR_DECL
     Cursor zc;
     zc.init(it0, p.units);
     int cur_head = -1;
-    uint32_t s = 0, ph = 0, j = 0, seg = 0;
+    uint32_t s = 0, ph = 0, j = 0, ub = 0, uph = 0, seg = 0;
     bool ok = true;
     for (; zc.it < it1 && ok; zc.next(p.units), ++j) {
       if (zc.major != cur_head) {
@@ -199,33 +210,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++seg;
         cur_head = zc.major;
       }
-      const uint32_t b = j & 1;
       TTT_TR_LAP(0);
       if (!(ok = mbar_wait_warp(&bars[BB_KE_FULL + s], ph, ab))) break;
       TTT_TR_LAP(1);
       const uint64_t soff = (s * L::kStage) >> 4;
       const uint64_t dk = dk0 + soff, de = de0 + soff;
-      // dA^T of this unit once the epilogue has read the previous one.
-      if (!(ok = mbar_wait_warp(&bars[BB_DA_EMPTY], (j & 1) ^ 1, ab))) break;
+      // U^T into buffer ub once the dW MMAs of unit j-3 have read it (early:
+      // this wait is off the critical path, so U goes first).
+      if (!(ok = mbar_wait_warp(&bars[BB_U_EMPTY + ub], uph ^ 1, ab))) break;
+      TTT_TR_LAP(5);
+      tc_fence_after();
+      const uint32_t tu = tbase + L::cU + ub * kUnit;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) mma_bf16_ts_warp(tu, tW1 + 8 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
+      // Z3^T and dA^T of this unit once the epilogue has read the previous ones.
+      if (!(ok = mbar_wait_warp(&bars[BB_ZD_EMPTY], (j & 1) ^ 1, ab))) break;
       TTT_TR_LAP(2);
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) mma_bf16_warp(tDA, dw2 + 2 * k, de + 2 * k, kId, k > 0 ? 1u : 0u);
-      // U^T, Z3^T into buffer b once the dW MMAs of unit j-2 have read it.
-      if (!(ok = mbar_wait_warp(&bars[BB_Z_EMPTY + b], ((j >> 1) & 1) ^ 1, ab))) break;
-      TTT_TR_LAP(5);
-      tc_fence_after();
-      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) mma_bf16_ts_warp(tz, tW + 8 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        mma_bf16_ts_warp(tz + kUnit, tW + D / 2 + 8 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
-      mma_commit_warp(&bars[BB_U_FULL + b]);
+      for (int k = 0; k < D / 16; ++k) mma_bf16_warp(tZ3, dw3 + 2 * k, dk + 2 * k, kId, k > 0 ? 1u : 0u);
+      mma_commit_warp(&bars[BB_FULL + ub]);
       TTT_TR_LAP(3);
       if (++s == kBwdStages) {
         s = 0;
         ph ^= 1;
+      }
+      if (++ub == kBwdUBufs) {
+        ub = 0;
+        uph ^= 1;
       }
     }
     TTT_TR_DUMP(2);
@@ -235,9 +249,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------ dW issuer
     // dW1^T += (2 dZ1^T) K, dW3^T += dZ3^T K, dW2 += A^T E per 16-token group
     // as soon as its epilogue warpgroup has written it.  The unit's last
-    // commits release its U/Z3 buffer and its K/E stage: the unit's other
-    // MMAs completed before the epilogue could read their results, so every
-    // reader of the stage is done.
+    // commits release its U buffer, its A^T slot and its K/E stage: the unit's
+    // other MMAs completed before the epilogue could read their results, so
+    // every reader of the stage is done.
     constexpr uint32_t kIdW = idesc_bf16(128, D, false, true);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
     const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
@@ -245,9 +259,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     TTT_TR_DECL
     Cursor wc;
     wc.init(it0, p.units);
-    uint32_t s = 0, j = 0, seg = 0;
+    uint32_t s = 0, ub = 0, uph = 0, pa = 0, seg = 0;
     bool ok = true;
-    for (; wc.it < it1 && ok; wc.next(p.units), ++j) {
+    for (; wc.it < it1 && ok; wc.next(p.units)) {
       const bool first = (wc.it == it0) || wc.tile == 0;
       const bool last = (wc.it == it1 - 1) || wc.tile == p.units - 1;
       if (first && seg > 0) {
@@ -255,31 +269,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!(ok = mbar_wait_warp(&bars[BB_ACC_EMPTY], (seg - 1) & 1, ab))) break;
         TTT_TR_LAP(4);
       }
-      const uint32_t b = j & 1;
-      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit);
+      const uint32_t tu = tbase + L::cU + ub * kUnit, tpa = tbase + L::cPA + pa * 24;
       const uint64_t soff = (s * L::kStage) >> 4;
       const uint64_t dk = dk0 + soff, de = de0 + soff;
 #pragma unroll
       for (int g = 0; g < 3; ++g) {
         TTT_TR_LAP(0);
-        if (!(ok = mbar_wait_warp(&bars[BB_P_FULL + 3 * b + g], (j >> 1) & 1, ab))) break;
+        if (!(ok = mbar_wait_warp(&bars[BB_P_FULL + 3 * ub + g], uph, ab))) break;
         TTT_TR_LAP(1);
         tc_fence_after();
         const uint32_t acc = (first && g == 0) ? 0u : 1u;
         const uint64_t go = (16u * g * SW) >> 4;
-        mma_bf16_ts_warp(tDW, tz + 16 * g, dk + go, kIdW, acc);
-        mma_bf16_ts_warp(tDW + D, tz + 16 * g + 8, dk + go, kIdW, acc);
-        mma_bf16_ts_warp(tDW + 2 * D, tz + kUnit + 16 * g, de + go, kIdW, acc);
+        mma_bf16_ts_warp(tDW, tu + 16 * g, dk + go, kIdW, acc);
+        mma_bf16_ts_warp(tDW + D, tu + 16 * g + 8, dk + go, kIdW, acc);
+        mma_bf16_ts_warp(tDW + 2 * D, tpa + 8 * g, de + go, kIdW, acc);
         TTT_TR_LAP(2);
       }
       if (!ok) break;
-      mma_commit_warp(&bars[BB_Z_EMPTY + b]);
+      mma_commit_warp(&bars[BB_U_EMPTY + ub]);
+      mma_commit_warp(&bars[BB_PA_EMPTY + pa]);
       mma_commit_warp(&bars[BB_KE_EMPTY + s]);
       if (last) {
         mma_commit_warp(&bars[BB_ACC_FULL]);   // segment done: the epilogue dumps dW
         ++seg;
       }
       if (++s == kBwdStages) s = 0;
+      if (++ub == kBwdUBufs) {
+        ub = 0;
+        uph ^= 1;
+      }
+      pa ^= 1;
     }
     TTT_TR_DUMP(2);
     mma_commit_warp(&bars[BB_DONE]);
@@ -290,7 +309,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int q = warp & 3;                    // TMEM lane quadrant
     const int row = q * 32 + lane;             // hidden unit within the slice
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t j = 0, seg = 0, dumps = 0;
+    uint32_t j = 0, ub = 0, uph = 0, seg = 0, dumps = 0;
     long long cur_pair = -1;
     bool ok = true;
     TTT_TR_DECL
@@ -325,17 +344,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       return true;
     };
 
-    // Weights of a (head, slice): warpgroup 0 writes W1^T/2 rows and warpgroup
-    // 1 W3^T rows into TMEM, warpgroup 2 the W2 rows into shared memory (the
-    // K-major, swizzled A operand of dA^T).
+    // Weights of a (head, slice): warpgroup 0 writes the W1^T/2 rows into TMEM,
+    // warpgroups 1 and 2 the W3^T and W2 rows into shared memory (the K-major,
+    // swizzled A operands of Z3^T and dA^T).
     auto load_weights = [&](int head) -> bool {
       if (seg > 0 && !mbar_wait(&bars[BB_W_EMPTY], (seg - 1) & 1, ab)) return false;
       tc_fence_after();
       const size_t hidp = static_cast<size_t>(p.slices) * 128;
       const uint4* src = reinterpret_cast<const uint4*>(
           p.wt_img + ((static_cast<size_t>(head) * hidp + slice_id * 128 + row) * 3 + g) * (D / 2));
-      if (g == 2) {
-        const uint32_t base = smem_u32(smem + L::off_w2);
+      if (g > 0) {
+        const uint32_t base = smem_u32(smem + (g == 1 ? L::off_w3 : L::off_w2));
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
           const uint4 x = __ldg(src + c);
@@ -351,7 +370,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint4 x = __ldg(src + c0 / 4 + v);
             w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
           }
-          tmem_st16(tbase + L::cW + g * (D / 2) + c0 + lane_off, w);
+          tmem_st16(tbase + L::cW1 + c0 + lane_off, w);
         }
         tmem_wait_st();
       } else {
@@ -361,7 +380,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint4 x = __ldg(src + v);
           w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
         }
-        tmem_st8(tbase + L::cW + g * (D / 2) + lane_off, w);
+        tmem_st8(tbase + L::cW1 + lane_off, w);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -380,22 +399,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!(ok = load_weights(cu.major))) break;
         cur_pair = pair;
       }
-      const uint32_t b = j & 1;
+      const uint32_t pa = j & 1;
       TTT_TR_LAP(0);
-      if (!(ok = mbar_wait(&bars[BB_U_FULL + b], (j >> 1) & 1, ab))) break;
+      if (!(ok = mbar_wait(&bars[BB_FULL + ub], uph, ab))) break;
       TTT_TR_LAP(1);
       tc_fence_after();
       uint32_t zu[16], z3[16], da[16];
-      const uint32_t tz = tbase + L::cZ + b * (2 * kUnit) + 16 * g + lane_off;
-      tmem_ld16(tz, zu);
-      tmem_ld16(tz + kUnit, z3);
+      const uint32_t tu = tbase + L::cU + ub * kUnit + 16 * g + lane_off;
+      // The single-buffered Z3^T / dA^T columns first: the next unit's MMAs
+      // into them wait for this release.
+      tmem_ld16(tbase + L::cZ3 + 16 * g + lane_off, z3);
       tmem_ld16(tbase + L::cDA + 16 * g + lane_off, da);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[BB_DA_EMPTY]);
+      if (lane == 0) mbar_arrive(&bars[BB_ZD_EMPTY]);
+      tmem_ld16(tu, zu);
+      tmem_wait_ld();
       TTT_TR_LAP(2);
-      uint32_t pz1[8], pz3[8], pa[8];
+      uint32_t pz1[8], pz3[8], pav[8];
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
         // Packed bf16 arithmetic on two tokens of this hidden unit (the outputs
@@ -412,18 +434,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t q2 = bfma2(bu, om, s2);                          // 2 dsilu/dz1
         pz1[i / 2] = bmul2(bmul2(bd, b3), q2);
         pz3[i / 2] = bmul2(bd, silu);
-        pa[i / 2] = bmul2(silu, b3);
+        pav[i / 2] = bmul2(silu, b3);
       }
       TTT_TR_LAP(3);
-      // Over the U/Z3 columns of this warpgroup's tokens, already read above.
-      tmem_st8(tz, pz1);
-      tmem_st8(tz + 8, pz3);
-      tmem_st8(tz + kUnit, pa);
+      // 2 dZ1^T, dZ3^T over this warpgroup's U columns (read above); A^T into
+      // its slot once the dW MMAs of unit j-2 have read it.
+      tmem_st8(tu, pz1);
+      tmem_st8(tu + 8, pz3);
+      if (!(ok = mbar_wait(&bars[BB_PA_EMPTY + pa], ((j >> 1) & 1) ^ 1, ab))) break;
+      TTT_TR_LAP(4);
+      tc_fence_after();
+      tmem_st8(tbase + L::cPA + pa * 24 + 8 * g + lane_off, pav);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[BB_P_FULL + 3 * b + g]);
+      if (lane == 0) mbar_arrive(&bars[BB_P_FULL + 3 * ub + g]);
       TTT_TR_LAP(7);
+      if (++ub == kBwdUBufs) {
+        ub = 0;
+        uph ^= 1;
+      }
     }
     if (ok && cur_pair >= 0) dump(cur_pair);
     TTT_TR_LAP(0);
