@@ -124,7 +124,8 @@ int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t*
  * that has already handed all device memory to a pool it does not control.
  * The paper has no counterpart of this entry point; it is a packaging
  * convenience.  It takes no workspace: its scratch (the status word and the
- * bf16 fast-weight images) lives in a fixed array of TTT_NOALLOC_SCRATCH_BYTES
+ * fast-weight operand images, bf16 W1/W3 and f16 W2) lives in a fixed array of
+ * TTT_NOALLOC_SCRATCH_BYTES
  * bytes that is part of the library, which every GPU that loads the library
  * holds until the process exits.  Shapes whose scratch would exceed it
  * (ttt_workspace_bytes(dims, TTT_OP_READ) > TTT_NOALLOC_SCRATCH_BYTES) return
