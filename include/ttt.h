@@ -36,10 +36,17 @@
  * a workspace clears when it starts, and are reported by ttt_check_status as
  * TTT_EDEVICE.
  *
- * Supported shapes: d in {16, 32, 64}; 1 <= h <= 256 (padded internally to a
- * multiple of 128 with zero weights, which is exact); heads >= 1;
- * grid_h, grid_w >= 1; 0 <= n_special; n >= 1.  Other shapes return
- * TTT_EUNSUPPORTED.
+ * Supported shapes: heads >= 1; grid_h, grid_w >= 1; 0 <= n_special; n >= 1;
+ * and either
+ *   d in {16, 32, 64} and 1 <= h <= 256 (padded internally to a multiple of
+ *   128 with zero weights, which is exact): the fused tensor-core kernels; or
+ *   d and h multiples of 64 (d <= 8192, h <= 32768), e.g. d = 1024, h = 2048:
+ *   the wide-head path, which runs the products as bf16 cuBLAS GEMMs with FP32
+ *   accumulation over chunks of 131072 tokens.  Its first call on a device
+ *   creates that device's cuBLAS handle (cuBLAS allocates its own small state
+ *   then); the GEMMs use the workspace for their scratch.  Calls of the wide
+ *   path on one device are serialised while they enqueue.
+ * Other shapes return TTT_EUNSUPPORTED.
  */
 #ifndef TTT_H_
 #define TTT_H_

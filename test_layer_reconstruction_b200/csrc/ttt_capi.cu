@@ -1,7 +1,11 @@
 // ttt_capi.cu — the C ABI declared in include/ttt.h: host-side validation,
 // workspace layout, TMA descriptors and the launch sequence of the layer
 //   conv -> steps x [pack theta -> forward (residual) -> backward (partials)
-//   -> reduce + SGD] -> pack theta* -> forward (read).
+//   -> reduce + SGD] -> pack theta* -> forward (read)
+// for head widths 16, 32, 64 (h <= 256), and the wide-head sequence (token
+// chunks of bf16 library GEMMs and the elementwise kernels of wide.cuh) for
+// head widths and hidden widths that are multiples of 64 beyond that.
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -14,27 +18,35 @@
 #include "../../include/ttt.h"
 #include "conv.cuh"
 #include "update.cuh"
+#include "wide.cuh"
 
 using namespace ttt;
 
 namespace {
 
 constexpr size_t kAlign = 1024;
+constexpr int kMaxDevicesWide = 64;
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
 struct Shape {
   long long n;   // tokens
   int H, D, h, hidp, tiles, slices, units;
   long long C;   // H * D channels
+  bool wide;     // wide-head path (library GEMMs over token chunks)
 };
+
+constexpr long long kWideChunk = 131072;           // tokens per GEMM chunk of the wide path
+constexpr size_t kWideGemmWorkspace = 32u << 20;   // library GEMM workspace (bytes)
 
 int check_dims(const ttt_dims* dm, Shape* s) {
   if (!dm) return TTT_EINVAL;
   if (dm->n_views < 1 || dm->grid_h < 1 || dm->grid_w < 1 || dm->n_special < 0 || dm->heads < 1 || dm->d < 1 ||
       dm->h < 1)
     return TTT_EINVAL;
-  if (!(dm->d == 16 || dm->d == 32 || dm->d == 64)) return TTT_EUNSUPPORTED;
-  if (dm->h > 256) return TTT_EUNSUPPORTED;
+  const bool fused = (dm->d == 16 || dm->d == 32 || dm->d == 64) && dm->h <= 256;
+  const bool wide = dm->d % 64 == 0 && dm->h % 64 == 0 && dm->d <= 8192 && dm->h <= 32768;
+  if (!fused && !wide) return TTT_EUNSUPPORTED;
+  s->wide = !fused;
   const long long T = static_cast<long long>(dm->n_special) + static_cast<long long>(dm->grid_h) * dm->grid_w;
   const long long n = T * dm->n_views;
   if (n <= 0 || n > (1LL << 31) - 1 - 128) return TTT_EUNSUPPORTED;   // TMA coordinates are int32
@@ -84,6 +96,7 @@ Grids grids_for(const Shape& s, int sms) {
 
 struct Ws {
   size_t status, w13, w2h, wt, vp, e, part, q, k, v, o, convw, th0, thout, total;
+  size_t img, acc, z1, z3, da, ab, eb, gemm;   // wide path
 };
 
 Ws ws_layout(const Shape& s, const Grids& g, int op) {
@@ -98,6 +111,32 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
   const size_t tok_bytes = static_cast<size_t>(s.n) * s.C * 2;
   const size_t theta_bytes = 3ull * s.H * s.D * s.h * 4;
   w.status = take(256);
+  if (s.wide) {
+    const bool writes = op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST;
+    const size_t nc = static_cast<size_t>(std::min<long long>(s.n, kWideChunk));
+    w.img = take(3ull * s.H * s.D * s.h * 2);
+    w.z1 = take(nc * s.h * 2);
+    w.z3 = take(nc * s.h * 2);
+    w.ab = take(nc * s.h * 2);
+    w.gemm = take(kWideGemmWorkspace);
+    if (writes) {
+      w.acc = take(3ull * s.D * s.h * 4);
+      w.da = take(nc * s.h * 2);
+      w.eb = take(nc * s.D * 2);
+      w.vp = take(tok_bytes);
+    }
+    if (op == TTT_OP_LAYER_HOST) {
+      w.q = take(tok_bytes);
+      w.k = take(tok_bytes);
+      w.v = take(tok_bytes);
+      w.o = take(tok_bytes);
+      w.convw = take(static_cast<size_t>(s.C) * 9 * 4);
+      w.th0 = take(theta_bytes);
+      w.thout = take(theta_bytes);
+    }
+    w.total = off;
+    return w;
+  }
   w.w13 = take(static_cast<size_t>(s.H) * 2 * s.hidp * s.D * 2);
   w.w2h = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
   if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST) {
@@ -317,9 +356,173 @@ int prepare(const ttt_dims* dm, int op, void* workspace, size_t ws_bytes, void* 
   return TTT_OK;
 }
 
+// ------------------------------------------------------------------ wide path
+// One library GEMM handle per device, created on first use; enqueues of the
+// wide path on a device are serialised because the handle's stream and
+// workspace are set per call.
+struct WideGemm {
+  std::mutex mu;
+  cublasHandle_t h[kMaxDevicesWide] = {};
+};
+WideGemm& wide_gemm() {
+  static WideGemm g;
+  return g;
+}
+
+// Row-major C[M x N] (ldc) = alpha op(A)[M x K] op(B)[K x N] + beta C, bf16 A and
+// B, FP32 accumulation; op(A) = A^T when `ta` (A stored K x M), likewise B.
+// Column-major view: C^T = op(B)^T op(A)^T.
+bool gemm_rm(cublasHandle_t hd, bool ta, bool tb, int M, int N, int K, float alpha, const void* A, int lda,
+             const void* B, int ldb, float beta, void* C, cudaDataType_t ctype, int ldc) {
+  return cublasGemmEx(hd, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, B,
+                      CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda, &beta, C, ctype, ldc, CUBLAS_COMPUTE_32F,
+                      CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
+}
+
+unsigned elementwise_grid(long long n8) {
+  const int sms = num_sms();
+  return static_cast<unsigned>(std::max<long long>(1, std::min<long long>((n8 + 255) / 256, 8LL * (sms > 0 ? sms : 148))));
+}
+
+// Takes the device's GEMM handle (created on first use) bound to this call's
+// stream and workspace; holds the device's lock for the caller's enqueue.
+struct WideCall {
+  std::unique_lock<std::mutex> lock;
+  cublasHandle_t hd = nullptr;
+  bool ok = false;
+  WideCall(const Call& c) : lock(wide_gemm().mu) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesWide) return;
+    cublasHandle_t& h = wide_gemm().h[dev];
+    if (!h && cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) {
+      h = nullptr;
+      return;
+    }
+    if (cublasSetStream(h, c.st) != CUBLAS_STATUS_SUCCESS) return;
+    if (cublasSetWorkspace(h, c.ws + c.w.gemm, kWideGemmWorkspace) != CUBLAS_STATUS_SUCCESS) return;
+    hd = h;
+    ok = true;
+  }
+};
+
+int wide_cast(const Call& c, const float* theta) {
+  const long long count = 3LL * c.s.H * c.s.D * c.s.h;
+  wide_cast_kernel<<<elementwise_grid(count / 8), 256, 0, c.st>>>(
+      theta, reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.img), count);
+  return launch_status();
+}
+
+// Z1, Z3 (bf16) of rows [t0, t0 + nc) of head hd of X, then A = silu(Z1) Z3.
+int wide_forward_chunk(const Call& c, cublasHandle_t hd, const uint16_t* X, int head, long long t0, int nc) {
+  const Shape& s = c.s;
+  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
+  const uint16_t* xc = X + (static_cast<size_t>(t0) * s.H + head) * s.D;
+  const int ldx = s.H * s.D;
+  if (!gemm_rm(hd, false, false, nc, s.h, s.D, 1.f, xc, ldx, img + head * per, s.h, 0.f, c.ws + c.w.z1, CUDA_R_16BF,
+               s.h) ||
+      !gemm_rm(hd, false, false, nc, s.h, s.D, 1.f, xc, ldx, img + (s.H + head) * per, s.h, 0.f, c.ws + c.w.z3,
+               CUDA_R_16BF, s.h))
+    return TTT_ECUDA;
+  const long long n8 = static_cast<long long>(nc) * s.h / 8;
+  wide_gate_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<const uint4*>(c.ws + c.w.z1),
+                                                           reinterpret_cast<const uint4*>(c.ws + c.w.z3),
+                                                           reinterpret_cast<uint4*>(c.ws + c.w.ab), n8);
+  return launch_status();
+}
+
+// The write of the wide path: per step, per head, per token chunk
+//   Z1, Z3, A (forward) -> E = A W2 - V' -> dA = E W2^T -> dZ1, dZ3
+//   -> dW1 += K^T dZ1, dW3 += K^T dZ3, dW2 += A^T E   (FP32, Eq. 5)
+// then theta_out = theta_in - lr (2/n) dW for the head.
+int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
+                   const float* theta0, float lr, int steps, float* theta_out) {
+  const Shape& s = c.s;
+  uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
+  if (rc != TTT_OK) return rc;
+  if (steps == 0) {
+    if (theta_out != theta0 &&
+        cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    return TTT_OK;
+  }
+  WideCall wc(c);
+  if (!wc.ok) return TTT_ECUDA;
+  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
+  float* acc = reinterpret_cast<float*>(c.ws + c.w.acc);
+  uint8_t* eb = c.ws + c.w.eb;
+  const int ldx = s.H * s.D;
+  const float scale = lr * 2.0f / static_cast<float>(s.n);
+  for (int step = 0; step < steps; ++step) {
+    const float* th_in = step == 0 ? theta0 : theta_out;
+    if ((rc = wide_cast(c, th_in)) != TTT_OK) return rc;
+    for (int head = 0; head < s.H; ++head) {
+      const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;   // [h][D]
+      for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
+        const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
+        const float beta = t0 == 0 ? 0.f : 1.f;
+        if ((rc = wide_forward_chunk(c, wc.hd, K, head, t0, nc)) != TTT_OK) return rc;
+        // E = A W2 - V' (the chunk's V' rows first copied into E)
+        if (cudaMemcpy2DAsync(eb, static_cast<size_t>(s.D) * 2, vp + (static_cast<size_t>(t0) * s.H + head) * s.D,
+                              static_cast<size_t>(ldx) * 2, static_cast<size_t>(s.D) * 2, nc,
+                              cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+          return TTT_ECUDA;
+        if (!gemm_rm(wc.hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, -1.f, eb, CUDA_R_16BF,
+                     s.D) ||
+            !gemm_rm(wc.hd, false, true, nc, s.h, s.D, 1.f, eb, s.D, w2, s.D, 0.f, c.ws + c.w.da, CUDA_R_16BF, s.h))
+          return TTT_ECUDA;
+        const long long n8 = static_cast<long long>(nc) * s.h / 8;
+        wide_dz_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<uint4*>(c.ws + c.w.z1),
+                                                               reinterpret_cast<uint4*>(c.ws + c.w.z3),
+                                                               reinterpret_cast<const uint4*>(c.ws + c.w.da), n8);
+        if ((rc = launch_status()) != TTT_OK) return rc;
+        const uint16_t* kc = K + (static_cast<size_t>(t0) * s.H + head) * s.D;
+        if (!gemm_rm(wc.hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z1, s.h, beta, acc, CUDA_R_32F,
+                     s.h) ||
+            !gemm_rm(wc.hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z3, s.h, beta, acc + per,
+                     CUDA_R_32F, s.h) ||
+            !gemm_rm(wc.hd, true, false, s.h, s.D, nc, 1.f, c.ws + c.w.ab, s.h, eb, s.D, beta, acc + 2 * per,
+                     CUDA_R_32F, s.D))
+          return TTT_ECUDA;
+      }
+      wide_sgd_kernel<<<elementwise_grid(static_cast<long long>(3 * per) / 8), 256, 0, c.st>>>(
+          th_in, theta_out, acc, s.H, s.D, s.h, head, scale);
+      if ((rc = launch_status()) != TTT_OK) return rc;
+    }
+  }
+  return TTT_OK;
+}
+
+// The read of the wide path: per head and token chunk, Z1, Z3, A, then
+// O = A W2 written straight into the head's columns of O.
+int run_read_wide(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
+  const Shape& s = c.s;
+  WideCall wc(c);
+  if (!wc.ok) return TTT_ECUDA;
+  int rc = wide_cast(c, theta);
+  if (rc != TTT_OK) return rc;
+  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
+  const int ldx = s.H * s.D;
+  for (int head = 0; head < s.H; ++head) {
+    const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;
+    for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
+      const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
+      if ((rc = wide_forward_chunk(c, wc.hd, Q, head, t0, nc)) != TTT_OK) return rc;
+      if (!gemm_rm(wc.hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, 0.f,
+                   O + (static_cast<size_t>(t0) * s.H + head) * s.D, CUDA_R_16BF, ldx))
+        return TTT_ECUDA;
+    }
+  }
+  return TTT_OK;
+}
+
 int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
               const float* theta0, float lr, int steps, float* theta_out) {
   const Shape& s = c.s;
+  if (s.wide) return run_write_wide(c, dm, K, V, conv_w, theta0, lr, steps, theta_out);
   uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
   uint16_t* e = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
   unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
@@ -382,6 +585,7 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
 
 int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
   const Shape& s = c.s;
+  if (s.wide) return run_read_wide(c, Q, theta, O);
   int rc = run_pack(s, theta, c.w, c.ws, false, c.st);
   if (rc != TTT_OK) return rc;
   CUtensorMap tq;

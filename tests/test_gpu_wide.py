@@ -1,0 +1,101 @@
+"""GPU parity of the wide-head path (head widths and hidden widths that are
+multiples of 64 beyond the fused kernels' d <= 64, h <= 256), through the C ABI.
+
+* Two 128-wide heads with h=192 on a ragged grid: full oracle parity.
+* The 2000-view workload's shape (one head, d=1024, h=2048, lr 0.02, 2 steps)
+  on a 4-view subset: full oracle parity.
+* 200 views of that shape (three 131072-token GEMM chunks): the chunk
+  accumulation checked by the Eq. 5 property delta(all) = sum_parts
+  (n_part/n) delta(part) at a step size where one step is far above the f32
+  resolution of theta, and bitwise determinism.
+* The full 2000-view layer plus the read of 200 held-out views with the
+  frozen theta*: rows of both outputs sampled against the oracle read with the
+  GPU's theta*.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ttt_oracle as orc
+from test_layer_reconstruction_b200 import inputs as tin
+from test_layer_reconstruction_b200 import ttt
+from ttt_testlib import (TOL_DELTA, TOL_O, TOL_THETA, bf16_inputs, compare_O, compare_theta, normwise,
+                         oracle_layer, to_device)
+
+pytestmark = pytest.mark.gpu
+
+BIG = tin.CONFIGS["views2000_37x37p5_h1_d1024_h2048"]
+
+
+def test_wide_small_heads_match_oracle():
+    cfg = tin.LayerConfig("wide_small", 3, 9, 11, 2, 2, 128, 192, 2, 0.1, 21)
+    inp = bf16_inputs(tin.make_inputs(cfg))
+    dev = to_device(inp)
+    theta, O = ttt.layer(dev["Q"], dev["K"], dev["V"], dev["conv_w"], dev["theta"], cfg.lr, cfg.steps, cfg)
+    torch.cuda.synchronize()
+    ref = oracle_layer(cfg, inp)
+    t_err, d_err = compare_theta(cfg, inp, theta, ref)
+    assert t_err <= TOL_THETA and d_err <= TOL_DELTA, (t_err, d_err)
+    assert compare_O(O, ref) <= TOL_O
+
+
+def test_views2000_shape_on_a_view_subset_matches_oracle():
+    cfg = BIG.with_views(4)
+    inp = bf16_inputs(tin.make_inputs(cfg))
+    dev = to_device(inp)
+    theta, O = ttt.layer(dev["Q"], dev["K"], dev["V"], dev["conv_w"], dev["theta"], cfg.lr, cfg.steps, cfg)
+    torch.cuda.synchronize()
+    ref = oracle_layer(cfg, inp)
+    t_err, d_err = compare_theta(cfg, inp, theta, ref)
+    assert t_err <= TOL_THETA and d_err <= TOL_DELTA, (t_err, d_err)
+    assert compare_O(O, ref) <= TOL_O
+
+
+def test_wide_chunk_accumulation_linearity_and_determinism():
+    """One SGD step is delta = -lr grad L(theta0), linear in lr; at lr = 20 the
+    step is far above the f32 resolution of theta, so the check isolates the
+    GEMM chunking (three chunks over 200 views, one or two over each part)."""
+    cfg = tin.LayerConfig(BIG.name, 200, BIG.grid_h, BIG.grid_w, BIG.n_special, 1, 1024, 2048, 1, 20.0, BIG.seed)
+    inp = tin.make_inputs(cfg, device="cuda")
+    K = inp["K"].to(torch.bfloat16).contiguous()
+    V = inp["V"].to(torch.bfloat16).contiguous()
+    w = inp["conv_w"].contiguous()
+    th0 = tin.pack_theta(inp["W1"], inp["W3"], inp["W2"]).cuda()
+    del inp
+    full = ttt.write(K, V, w, th0, cfg.lr, 1, cfg)
+    again = ttt.write(K, V, w, th0, cfg.lr, 1, cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(full, again)
+    T = cfg.tokens_per_view
+    acc = torch.zeros_like(full, dtype=torch.float64)
+    for a, b in ((0, 90), (90, 200)):
+        part = cfg.with_views(b - a)
+        th = ttt.write(K[a * T:b * T].contiguous(), V[a * T:b * T].contiguous(), w, th0, cfg.lr, 1, part)
+        torch.cuda.synchronize()
+        acc += (th.double() - th0.double()) * ((b - a) / cfg.n_views)
+    delta = (full.double() - th0.double()).cpu().numpy()
+    assert normwise(acc.cpu().numpy(), delta) <= 5e-4
+
+
+def test_views2000_layer_and_heldout_read_sampled_rows():
+    cfg = BIG
+    inp = tin.make_inputs(cfg, device="cuda")
+    Q, K, V = (inp[k].to(torch.bfloat16).contiguous() for k in ("Q", "K", "V"))
+    w = inp["conv_w"].contiguous()
+    W = (inp["W1"].cpu(), inp["W3"].cpu(), inp["W2"].cpu())
+    th0 = tin.pack_theta(*W).cuda()
+    del inp
+    torch.cuda.empty_cache()
+    theta, O = ttt.layer(Q, K, V, w, th0, cfg.lr, cfg.steps, cfg)
+    held = tin.make_inputs(cfg, device="cuda", heldout=True)["Q"].to(torch.bfloat16).contiguous()
+    O_held = ttt.read(held, theta, cfg.with_views(cfg.heldout_views))
+    torch.cuda.synchronize()
+    W1g, W3g, W2g = (t[0].double().numpy() for t in tin.unpack_theta(theta.cpu(), 1, cfg.d, cfg.h))
+    assert np.isfinite(W1g).all() and np.isfinite(W2g).all()
+    d_norm = max(np.abs(W1g - W[0][0].double().numpy()).max(), np.abs(W2g - W[2][0].double().numpy()).max())
+    assert d_norm > 0                                       # the write moved theta
+    g = np.random.default_rng(7)
+    for X, Y in ((Q, O), (held, O_held)):
+        rows = g.choice(X.shape[0], 512, replace=False)
+        ref = orc.read(X[rows, 0].double().cpu().numpy(), W1g, W3g, W2g)
+        assert normwise(Y[rows, 0].float().cpu().numpy(), ref) <= TOL_O
