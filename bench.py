@@ -316,6 +316,55 @@ def run_ours(args, cfg):
                "wall_s_per_step": (time.perf_counter() - t0) / args.e2e_steps}
         del ws_h
 
+    # Linear-scaling sweep over view counts (prefixes of the same inputs: views
+    # are contiguous token ranges) and the write-only / read-only split at 100
+    # views, each timed with CUDA events like the main run.
+    sweep, paths = None, None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        T = cfg.tokens_per_view
+
+        def time_calls(fn, reps=3, warm=2):
+            for _ in range(warm):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+
+        pts = []
+        for v in (100, 250, 500):
+            if v >= cfg.n_views:
+                continue
+            sub, nt = cfg.with_views(v), v * T
+            q, k, vv = Q[:nt], K[:nt], V[:nt]
+            th, o = torch.empty_like(theta0), torch.empty_like(q)
+            wsv = ttt.make_workspace(sub, ttt.OP_LAYER)
+            ms_v = time_calls(lambda: ttt.layer(q, k, vv, conv_w, theta0, cfg.lr, cfg.steps, sub, theta_out=th, O=o,
+                                                workspace=wsv))
+            pts.append((v, ms_v))
+            if ttt.check_status(wsv) != 0:
+                raise SystemExit(f"device status word set during the {v}-view sweep point")
+            del wsv
+        pts.append((cfg.n_views, ms_max))
+        sweep = {"views": [v for v, _ in pts], "ms_per_call": [round(m, 3) for _, m in pts],
+                 "tokens_per_s": [v * T / (m / 1e3) for v, m in pts]}
+        v = min(100, cfg.n_views)
+        sub, nt = cfg.with_views(v), v * T
+        q, k, vv = Q[:nt], K[:nt], V[:nt]
+        th, o = torch.empty_like(theta0), torch.empty_like(q)
+        wsw, wsr = ttt.make_workspace(sub, ttt.OP_WRITE), ttt.make_workspace(sub, ttt.OP_READ)
+        ms_w = time_calls(lambda: ttt.write(k, vv, conv_w, theta0, cfg.lr, cfg.steps, sub, theta_out=th, workspace=wsw))
+        ms_r = time_calls(lambda: ttt.read(q, th, sub, O=o, workspace=wsr))
+        paths = {"views": v, "write_ms": round(ms_w, 3), "write_tokens_per_s": nt / (ms_w / 1e3),
+                 "read_ms": round(ms_r, 3), "read_tokens_per_s": nt / (ms_r / 1e3)}
+        if ttt.check_status(wsw) != 0 or ttt.check_status(wsr) != 0:
+            raise SystemExit("device status word set during the write/read split")
+        del wsw, wsr
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, _ = _oracle_tokens_per_s(cfg, args.cpu_seconds)
@@ -328,10 +377,10 @@ def run_ours(args, cfg):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg.name, "n_views": cfg.n_views, "tokens": cfg.n, "heads": cfg.heads,
                        "d": cfg.d, "h": cfg.h, "steps": cfg.steps, "lr": cfg.lr,
-                       "l2": "no flush: every token tensor (2.8 GB) exceeds the 126 MB L2",
+                       "l2": f"no flush: every token tensor ({cfg.n * cfg.heads * cfg.d * 2 / 1e9:.2f} GB) exceeds the 126 MB L2",
                        "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": gpu_launches, "clocks": clk,
+            "gpu_launches": gpu_launches, "clocks": clk, "sweep": sweep, "paths": paths,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -339,32 +388,32 @@ def run_ours(args, cfg):
     return 0
 
 
-def _kernel_source_digest() -> str:
-    """sha256 over the CUDA sources (csrc/*.cu, csrc/*.cuh, by name)."""
+def _source_digest(files) -> str:
+    """sha256 over the named CUDA sources (test_layer_reconstruction_b200/csrc), in the given order."""
     import hashlib
     d = os.path.join(ROOT, "test_layer_reconstruction_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(name.encode())
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(f.read())
+    for name in files:
+        h.update(name.encode())
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
 def _traffic_from_profiles(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary
-    (profiles/traffic.json), or None when the counters were taken on other
-    kernel sources or another workload."""
+    (profiles/traffic.json), or None when the counters were taken on another
+    workload or the kernel's sources have changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         with open(path) as f:
             t = json.load(f)
-        if t.get("source_sha256") != _kernel_source_digest() or t.get("workload") != workload:
+        e = t["kernels"].get(kernel)
+        if t.get("workload") != workload or e is None or e["sha256"] != _source_digest(e["sources"]):
             return None
-        return t["bytes_per_launch"].get(kernel)
+        return e["bytes_per_launch"]
     except Exception:
         return None
 
@@ -379,6 +428,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the view-count sweep and write/read split")
     args = ap.parse_args()
     from test_layer_reconstruction_b200 import inputs as tin
     cfg = tin.CONFIGS[args.config]
