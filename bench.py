@@ -140,6 +140,29 @@ def _oracle_tokens_per_s(cfg, seconds_budget: float):
 
 
 # ----------------------------------------------------------------------------- arms
+def replica_config(cfg, rank: int):
+    """The workload of `rank` in a multi-GPU run: the same shape, its own scene
+    (seed offset by rank)."""
+    from test_layer_reconstruction_b200 import inputs as tin
+    return tin.LayerConfig(cfg.name, cfg.n_views, cfg.grid_h, cfg.grid_w, cfg.n_special, cfg.heads, cfg.d, cfg.h,
+                           cfg.steps, cfg.lr, cfg.seed + 1000 * rank)
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks call it, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_rank: int, ms_max: float) -> float:
+    """All ranks' tokens over the slowest rank's time (weak scaling)."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -209,8 +232,7 @@ def run_ours(args, cfg):
             dist.barrier()
 
     # Each rank draws its own replica (seed offset by rank).
-    rcfg = tin.LayerConfig(cfg.name, cfg.n_views, cfg.grid_h, cfg.grid_w, cfg.n_special, cfg.heads, cfg.d, cfg.h,
-                           cfg.steps, cfg.lr, cfg.seed + 1000 * rank)
+    rcfg = replica_config(cfg, rank)
     inp = tin.make_inputs(rcfg, device="cuda")
     Q = inp["Q"].to(torch.bfloat16).contiguous()
     K = inp["K"].to(torch.bfloat16).contiguous()
@@ -250,11 +272,8 @@ def run_ours(args, cfg):
     ms = e0.elapsed_time(e1) / args.steps
     if ttt.check_status(ws) != 0:
         raise SystemExit("device status word set during the timed steps")
-    ms_t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    value = world * cfg.n / (ms_max / 1e3)
+    ms_max = max_over_ranks(ms, world, "cuda")
+    value = whole_job_tokens_per_s(world, cfg.n, ms_max)
 
     # per-kernel roofline from the live event timings
     peaks = _peaks()
@@ -308,10 +327,8 @@ def run_ours(args, cfg):
         f1.record(stream)
         torch.cuda.synchronize()
         e_ms = f0.elapsed_time(f1) / args.e2e_steps
-        e_t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * cfg.n / (float(e_t.item()) / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e_max = max_over_ranks(e_ms, world, "cuda")
+        e2e = {"value": whole_job_tokens_per_s(world, cfg.n, e_max), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "wall_s_per_step": (time.perf_counter() - t0) / args.e2e_steps}
         del ws_h
