@@ -22,8 +22,7 @@ Plain, slow, obviously-correct numpy in float64.  Pages cited below:
   is not enough: ShortConv2D is a depthwise 3x3 convolution applied within
   a single image only.
 
-Readings taken where the pages are silent or disagree (each one is listed in
-the design doc with its reason):
+Readings taken where the pages are silent or disagree:
 
 * Loss: mean over all n tokens (special tokens included) of ||T(k) - v'||^2.
 * Inner optimiser: plain SGD, theta <- theta - lr * grad, each step a
@@ -35,7 +34,7 @@ the design doc with its reason):
 
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against
 facts that do not come from this file (library routines, finite differences,
-closed forms, brute force, invariants); see the design doc for the list.
+closed forms, brute force, invariants).
 """
 from __future__ import annotations
 
