@@ -7,13 +7,22 @@
 // FP32 accumulation, bf16 round-to-nearest-even store.
 //
 // HBM-bound: every value is read once from DRAM and V' written once.  A
-// thread owns 4 channels (one 8-byte vector) of one grid row of one view and
-// sweeps the row left to right with a 3x3 window of vectors in registers, so
-// each input vector is fetched by three threads (rows y-1, y, y+1) through
-// L1/L2 and only once from DRAM.  A warp covers 32 consecutive vectors of a
-// token (256 contiguous bytes).  Columns x+1 and x+2 are in flight while
-// column x is computed; 4 channels per thread keep the weights to 36
-// registers so three 256-thread blocks fit per SM.
+// thread owns 4 channels (one 8-byte vector) of a band of kConvBand grid rows
+// of one view and sweeps the band left to right, reading the kConvBand + 2
+// input rows around it.  A warp covers 32 consecutive vectors of a token (256
+// contiguous bytes).
+//
+// What limits such a sweep is the number of bytes in flight per SM, not the
+// arithmetic: the threads of neighbouring bands request a shared row from L2
+// at about the same moment, so only part of the requests are new DRAM bytes.
+// Bands of 2 rows cut the requests per row from three to two, and each thread
+// streams its input columns through a private ring of kConvRing columns in
+// shared memory with cp.async (no registers held while a copy is in flight;
+// the thread reads back only what it copied itself, so cp.async.wait_group is
+// the only synchronisation).  The window lives in registers as FP32: columns
+// x-1, x, x+1 of the band's input rows; only the column that enters it is read
+// and unpacked, and the sweep is unrolled by three so the window's roles
+// rotate without register moves.
 #pragma once
 #include "sm100.cuh"
 
@@ -32,79 +41,134 @@ __device__ __forceinline__ void unpack4(const uint2& u, float (&f)[4]) {
   f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
 }
 
-// Persistent blocks: grid = (blocks, ceil(C/4 / blockDim.x)).  Block b walks
-// the items b, b + gridDim.x, ... of the (view, grid row) space, item row ==
-// grid_h meaning the view's special tokens.  A thread's 36 weights are loaded
-// once per block instead of once per row.
-__global__ void __launch_bounds__(kConvThreads, 3) shortconv_kernel(const ConvParams p) {
+constexpr int kConvRing = 8;   // columns in the per-thread shared-memory ring
+constexpr int kConvBand = 2;   // output rows per thread (3 no longer fits 128 registers)
+
+__host__ __device__ constexpr size_t conv_smem_bytes(int threads) {
+  return static_cast<size_t>(kConvRing) * (kConvBand + 2) * threads * sizeof(uint2);
+}
+
+// 8-byte asynchronous copy global -> shared; src_bytes == 0 writes zeros and
+// reads nothing (the address is then never dereferenced).
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Persistent blocks: grid = (blocks, ceil(C/4 / blockDim.x)).  A thread
+// computes a band of R output rows (y0 .. y0+R-1) from the R+2 input rows
+// around it, so a row is requested from L2 (R+2)/R times instead of three.
+// Block b walks the items b, b + gridDim.x, ... of the (view, band) space,
+// band == bands meaning the view's special tokens.  A thread's 36 weights are
+// loaded once per block instead of once per band.
+template <int R>
+__global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvParams p) {
+  constexpr int NR = R + 2;   // input rows of a band
+  extern __shared__ __align__(16) uint8_t conv_smem[];
   const int G4 = p.C / 4;
   const int cg = blockIdx.y * blockDim.x + threadIdx.x;
   if (cg >= G4) return;
   const long long T = static_cast<long long>(p.n_special) + static_cast<long long>(p.gh) * p.gw;
-  const long long items = static_cast<long long>(p.n_views) * (p.gh + 1);
+  const int bands = (p.gh + R - 1) / R;
+  const long long items = static_cast<long long>(p.n_views) * (bands + 1);
   float w[4][9];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
     for (int k = 0; k < 9; ++k) w[c][k] = __ldg(p.w + static_cast<size_t>(cg * 4 + c) * 9 + k);
-  const uint2 zero = make_uint2(0, 0);
+  // ring slot s, band row i of this thread: consecutive threads, consecutive 8 bytes
+  const uint32_t ring = smem_u32(conv_smem) + threadIdx.x * 8u;
+  const uint32_t row_stride = blockDim.x * 8u, slot_stride = NR * row_stride;
 
   for (long long item = blockIdx.x; item < items; item += gridDim.x) {
-    const int view = static_cast<int>(item / (p.gh + 1));
-    const int y = static_cast<int>(item % (p.gh + 1));
+    const int view = static_cast<int>(item / (bands + 1));
+    const int band = static_cast<int>(item % (bands + 1));
     const long long vbase = static_cast<long long>(view) * T;
-    if (y == p.gh) {
+    if (band == bands) {
       for (int s = 0; s < p.n_special; ++s) {
         const long long t = vbase + s;
         p.out[t * G4 + cg] = __ldg(p.V + t * G4 + cg);
       }
       continue;
     }
+    const int y0 = band * R;
     const long long gbase = vbase + p.n_special;  // first patch token of the view
-    const bool row_ok[3] = {y >= 1, true, y + 1 < p.gh};
-    auto ld = [&](int a, int xx) -> uint2 {
-      if (!row_ok[a] || xx >= p.gw) return zero;
-      return __ldg(p.V + (gbase + static_cast<long long>(y - 1 + a) * p.gw + xx) * G4 + cg);
+    bool row_ok[NR];
+    const uint2* rowp[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      const int yy = y0 - 1 + i;
+      row_ok[i] = yy >= 0 && yy < p.gh;
+      rowp[i] = p.V + (gbase + static_cast<long long>(row_ok[i] ? yy : y0) * p.gw) * G4 + cg;
+    }
+    uint2* outp = p.out + (gbase + static_cast<long long>(y0) * p.gw) * G4 + cg;
+    const long long out_row = static_cast<long long>(p.gw) * G4;
+    // column xx into its ring slot (zeros outside the grid), one commit group per column
+    auto fetch = [&](int xx) {
+      const uint32_t slot = ring + static_cast<uint32_t>(xx % kConvRing) * slot_stride;
+      const bool col_ok = xx < p.gw;
+#pragma unroll
+      for (int i = 0; i < NR; ++i)
+        if (row_ok[i] && col_ok) cp_async8(slot + i * row_stride, rowp[i] + static_cast<long long>(xx) * G4, 8u);
+      cp_async_commit();
     };
-    // columns x-1, x, x+1 of rows y-1, y, y+1, and x+2 in flight
-    uint2 c0[3], c1[3], c2[3], c3[3];
+    // column xx from its ring slot, unpacked (the caller waited for its group)
+    auto take = [&](int xx, float (&dst)[NR][4]) {
+      const uint32_t slot = ring + static_cast<uint32_t>(xx % kConvRing) * slot_stride;
 #pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      c0[a] = zero;
-      c1[a] = ld(a, 0);
-      c2[a] = ld(a, 1);
-      c3[a] = ld(a, 2);
-    }
-    for (int x = 0; x < p.gw; ++x) {
-      uint2 c4[3];
-#pragma unroll
-      for (int a = 0; a < 3; ++a) c4[a] = ld(a, x + 3);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        float f0[4], f1[4], f2[4];
-        unpack4(c0[a], f0);
-        unpack4(c1[a], f1);
-        unpack4(c2[a], f2);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          acc[c] = fmaf(w[c][3 * a + 0], f0[c], acc[c]);
-          acc[c] = fmaf(w[c][3 * a + 1], f1[c], acc[c]);
-          acc[c] = fmaf(w[c][3 * a + 2], f2[c], acc[c]);
-        }
+      for (int i = 0; i < NR; ++i) {
+        uint2 u = make_uint2(0u, 0u);
+        if (row_ok[i] && xx < p.gw)
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(u.x), "=r"(u.y) : "r"(slot + i * row_stride));
+        unpack4(u, dst[i]);
       }
-      uint2 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      p.out[(gbase + static_cast<long long>(y) * p.gw + x) * G4 + cg] = o;
+    };
+    // One output column x of the band from the window (L, M, R) = columns
+    // (x-1, x, x+1).  First the slot of column x-1 (read at least one step
+    // earlier) is refilled with column x+kConvRing-1; after the outputs,
+    // column x+2 replaces L (it becomes the right column of x+1's window).
+    // Pending then are columns x+2 .. x+kConvRing-1, so column x+2 is
+    // complete once at most kConvRing-3 groups remain.
+    auto step = [&](float (&L)[NR][4], float (&M)[NR][4], float (&Rt)[NR][4], int x) {
+      fetch(x + kConvRing - 1);
 #pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        c0[a] = c1[a];
-        c1[a] = c2[a];
-        c2[a] = c3[a];
-        c3[a] = c4[a];
+      for (int r = 0; r < R; ++r) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            acc[c] = fmaf(w[c][3 * a + 0], L[r + a][c], acc[c]);
+            acc[c] = fmaf(w[c][3 * a + 1], M[r + a][c], acc[c]);
+            acc[c] = fmaf(w[c][3 * a + 2], Rt[r + a][c], acc[c]);
+          }
+        uint2 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        if (y0 + r < p.gh) outp[r * out_row + static_cast<long long>(x) * G4] = o;
       }
+      cp_async_wait<kConvRing - 3>();
+      take(x + 2, L);
+    };
+    float fa[NR][4], fb[NR][4], fc[NR][4];
+    for (int xx = 0; xx < kConvRing - 1; ++xx) fetch(xx);   // columns 0 .. kConvRing-2
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) fa[i][c] = 0.f;   // column -1: zero padding
+    cp_async_wait<kConvRing - 3>();                 // columns 0 and 1 complete
+    take(0, fb);
+    take(1, fc);
+    for (int x = 0; x < p.gw; x += 3) {
+      step(fa, fb, fc, x);
+      if (x + 1 >= p.gw) break;
+      step(fb, fc, fa, x + 1);
+      if (x + 2 >= p.gw) break;
+      step(fc, fa, fb, x + 2);
     }
+    cp_async_wait<0>();   // no copy of this band may land in the next band's ring
   }
 }
 

@@ -256,12 +256,16 @@ int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float*
   p.C = static_cast<int>(s.C);
   const int g4 = p.C / 4;
   const int block = std::min(kConvThreads, (g4 + 31) / 32 * 32);
-  const long long items = static_cast<long long>(dm->n_views) * (dm->grid_h + 1);
+  const long long items = static_cast<long long>(dm->n_views) * ((dm->grid_h + kConvBand - 1) / kConvBand + 1);
   const int sms = num_sms();
-  const long long persistent = static_cast<long long>(sms > 0 ? sms : 148) * 3;
+  const long long persistent = static_cast<long long>(sms > 0 ? sms : 148) * 2;
   dim3 grid(static_cast<unsigned>(std::min(items, persistent)), (g4 + block - 1) / block, 1);
+  const size_t smem = conv_smem_bytes(block);
+  if (cudaFuncSetAttribute(shortconv_kernel<kConvBand>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return TTT_ECUDA;
   ProfScope prof(KK_CONV, st);
-  shortconv_kernel<<<grid, block, 0, st>>>(p);
+  shortconv_kernel<kConvBand><<<grid, block, smem, st>>>(p);
   return launch_status();
 }
 
