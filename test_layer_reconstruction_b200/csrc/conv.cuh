@@ -37,19 +37,37 @@ struct ConvParams {
   int n_views, gh, gw, n_special, C;
 };
 
-__device__ __forceinline__ void unpack4(const uint2& u, float (&f)[4]) {
-  f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+// Two FP32 lanes in one 64-bit register pair, for the packed f32x2 FMA of
+// sm_100 (two independent fma.rn.f32 per instruction, bitwise equal to them).
+__device__ __forceinline__ uint64_t f32x2_from_bf16x2(uint32_t v) {
+  uint64_t r;
+  asm("{ .reg .b32 l, h; shl.b32 l, %1, 16; and.b32 h, %1, 0xffff0000; mov.b64 %0, {l, h}; }" : "=l"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_fma(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint32_t bf16x2_from_f32x2(uint64_t v) {
+  uint32_t r;
+  asm("{ .reg .b32 l, h; mov.b64 {l, h}, %1; cvt.rn.bf16x2.f32 %0, h, l; }" : "=r"(r) : "l"(v));
+  return r;
 }
 
 constexpr int kConvRing = 8;   // columns in the per-thread shared-memory ring
-constexpr int kConvBand = 2;   // output rows per thread (3 no longer fits 128 registers)
+constexpr int kConvBand = 3;   // output rows per thread
+static_assert((kConvRing & (kConvRing - 1)) == 0, "ring slots are masked");
 
 __host__ __device__ constexpr size_t conv_smem_bytes(int threads) {
   return static_cast<size_t>(kConvRing) * (kConvBand + 2) * threads * sizeof(uint2);
 }
 
 // 8-byte asynchronous copy global -> shared; src_bytes == 0 writes zeros and
-// reads nothing (the address is then never dereferenced).
+// reads nothing.
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -73,11 +91,14 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
   const long long T = static_cast<long long>(p.n_special) + static_cast<long long>(p.gh) * p.gw;
   const int bands = (p.gh + R - 1) / R;
   const long long items = static_cast<long long>(p.n_views) * (bands + 1);
-  float w[4][9];
+  // weights of channel pairs (4cg, 4cg+1) and (4cg+2, 4cg+3), per tap
+  uint64_t wp[2][9];
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
+  for (int q = 0; q < 2; ++q)
 #pragma unroll
-    for (int k = 0; k < 9; ++k) w[c][k] = __ldg(p.w + static_cast<size_t>(cg * 4 + c) * 9 + k);
+    for (int k = 0; k < 9; ++k)
+      wp[q][k] = f32x2_make(__ldg(p.w + static_cast<size_t>(cg * 4 + 2 * q) * 9 + k),
+                            __ldg(p.w + static_cast<size_t>(cg * 4 + 2 * q + 1) * 9 + k));
   // ring slot s, band row i of this thread: consecutive threads, consecutive 8 bytes
   const uint32_t ring = smem_u32(conv_smem) + threadIdx.x * 8u;
   const uint32_t row_stride = blockDim.x * 8u, slot_stride = NR * row_stride;
@@ -95,34 +116,46 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
     }
     const int y0 = band * R;
     const long long gbase = vbase + p.n_special;  // first patch token of the view
-    bool row_ok[NR];
+    // rows outside the grid are fetched as zeros (source size 0) from row y0
+    uint32_t row_bytes[NR];
     const uint2* rowp[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
       const int yy = y0 - 1 + i;
-      row_ok[i] = yy >= 0 && yy < p.gh;
-      rowp[i] = p.V + (gbase + static_cast<long long>(row_ok[i] ? yy : y0) * p.gw) * G4 + cg;
+      const bool ok = yy >= 0 && yy < p.gh;
+      row_bytes[i] = ok ? 8u : 0u;
+      rowp[i] = p.V + (gbase + static_cast<long long>(ok ? yy : y0) * p.gw) * G4 + cg;
     }
+    bool out_ok[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) out_ok[r] = y0 + r < p.gh;
     uint2* outp = p.out + (gbase + static_cast<long long>(y0) * p.gw) * G4 + cg;
     const long long out_row = static_cast<long long>(p.gw) * G4;
-    // column xx into its ring slot (zeros outside the grid), one commit group per column
+    auto slot_of = [&](int xx) { return ring + (static_cast<uint32_t>(xx) & (kConvRing - 1)) * slot_stride; };
+    // column xx into its ring slot, one commit group per column (empty past the grid)
     auto fetch = [&](int xx) {
-      const uint32_t slot = ring + static_cast<uint32_t>(xx % kConvRing) * slot_stride;
-      const bool col_ok = xx < p.gw;
+      if (xx < p.gw) {
+        const uint32_t slot = slot_of(xx);
+        const long long off = static_cast<long long>(xx) * G4;
 #pragma unroll
-      for (int i = 0; i < NR; ++i)
-        if (row_ok[i] && col_ok) cp_async8(slot + i * row_stride, rowp[i] + static_cast<long long>(xx) * G4, 8u);
+        for (int i = 0; i < NR; ++i) cp_async8(slot + i * row_stride, rowp[i] + off, row_bytes[i]);
+      }
       cp_async_commit();
     };
-    // column xx from its ring slot, unpacked (the caller waited for its group)
-    auto take = [&](int xx, float (&dst)[NR][4]) {
-      const uint32_t slot = ring + static_cast<uint32_t>(xx % kConvRing) * slot_stride;
+    // column xx from its ring slot as FP32 pairs (the caller waited for its group)
+    auto take = [&](int xx, uint64_t (&dst)[NR][2]) {
+      if (xx < p.gw) {
+        const uint32_t slot = slot_of(xx);
 #pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        uint2 u = make_uint2(0u, 0u);
-        if (row_ok[i] && xx < p.gw)
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(u.x), "=r"(u.y) : "r"(slot + i * row_stride));
-        unpack4(u, dst[i]);
+        for (int i = 0; i < NR; ++i) {
+          uint32_t lo, hi;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(slot + i * row_stride));
+          dst[i][0] = f32x2_from_bf16x2(lo);
+          dst[i][1] = f32x2_from_bf16x2(hi);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) dst[i][0] = dst[i][1] = 0ull;
       }
     };
     // One output column x of the band from the window (L, M, R) = columns
@@ -130,35 +163,33 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
     // earlier) is refilled with column x+kConvRing-1; after the outputs,
     // column x+2 replaces L (it becomes the right column of x+1's window).
     // Pending then are columns x+2 .. x+kConvRing-1, so column x+2 is
-    // complete once at most kConvRing-3 groups remain.
-    auto step = [&](float (&L)[NR][4], float (&M)[NR][4], float (&Rt)[NR][4], int x) {
+    // complete once at most kConvRing-3 groups remain.  Per channel the taps
+    // are summed row by row, left to right.
+    auto step = [&](uint64_t (&L)[NR][2], uint64_t (&M)[NR][2], uint64_t (&Rt)[NR][2], int x) {
       fetch(x + kConvRing - 1);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
         for (int a = 0; a < 3; ++a)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            acc[c] = fmaf(w[c][3 * a + 0], L[r + a][c], acc[c]);
-            acc[c] = fmaf(w[c][3 * a + 1], M[r + a][c], acc[c]);
-            acc[c] = fmaf(w[c][3 * a + 2], Rt[r + a][c], acc[c]);
+          for (int q = 0; q < 2; ++q) {
+            f32x2_fma(acc[q], wp[q][3 * a + 0], L[r + a][q]);
+            f32x2_fma(acc[q], wp[q][3 * a + 1], M[r + a][q]);
+            f32x2_fma(acc[q], wp[q][3 * a + 2], Rt[r + a][q]);
           }
-        uint2 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        if (y0 + r < p.gh) outp[r * out_row + static_cast<long long>(x) * G4] = o;
+        if (out_ok[r])
+          outp[r * out_row + static_cast<long long>(x) * G4] = make_uint2(bf16x2_from_f32x2(acc[0]),
+                                                                          bf16x2_from_f32x2(acc[1]));
       }
       cp_async_wait<kConvRing - 3>();
       take(x + 2, L);
     };
-    float fa[NR][4], fb[NR][4], fc[NR][4];
+    uint64_t fa[NR][2], fb[NR][2], fc[NR][2];
     for (int xx = 0; xx < kConvRing - 1; ++xx) fetch(xx);   // columns 0 .. kConvRing-2
 #pragma unroll
-    for (int i = 0; i < NR; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) fa[i][c] = 0.f;   // column -1: zero padding
-    cp_async_wait<kConvRing - 3>();                 // columns 0 and 1 complete
+    for (int i = 0; i < NR; ++i) fa[i][0] = fa[i][1] = 0ull;   // column -1: zero padding
+    cp_async_wait<kConvRing - 3>();                              // columns 0 and 1 complete
     take(0, fb);
     take(1, fc);
     for (int x = 0; x < p.gw; x += 3) {
