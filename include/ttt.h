@@ -116,10 +116,18 @@ int ttt_layer(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const 
               void* stream);
 
 /* ttt_layer on HOST buffers: copies Q, K, V, conv_w, theta0 to device copies
- * inside the workspace (one cudaMemcpyAsync each), runs the layer, copies
- * theta* and O back to the host buffers, all on `stream`.  Returns once the
- * work is enqueued; the host outputs are valid after the stream
- * synchronises.  Pinned host memory makes the copies asynchronous.
+ * inside the workspace, runs the layer, and copies theta* and O back to the
+ * host buffers.  On the fused path the copies are pipelined: conv_w, theta0,
+ * V and K go up first; Q then follows in up to 8 chunks of whole 128-token
+ * tiles while the write runs; each chunk is read as soon as it has landed, and
+ * its O goes back while the next chunk is read.  The call creates two helper
+ * streams and their events, and destroys them before returning (CUDA
+ * releases them once their work has completed).  They start after the work
+ * enqueued earlier on `stream`, and `stream` waits for all of them, so the
+ * call behaves as if everything ran on `stream`.  The wide-head path copies in
+ * order on `stream`.  Returns once the work is enqueued; the host outputs are
+ * valid after the stream synchronises.  Pinned host memory makes the copies
+ * asynchronous and lets them overlap.
  * Workspace: ttt_workspace_bytes(dims, TTT_OP_LAYER_HOST). */
 int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t* K_host,
                    const uint16_t* V_host, const float* conv_w_host,

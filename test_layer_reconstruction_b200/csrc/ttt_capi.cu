@@ -587,11 +587,12 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   return TTT_OK;
 }
 
-int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
-  const Shape& s = c.s;
-  if (s.wide) return run_read_wide(c, Q, theta, O);
-  int rc = run_pack(s, theta, c.w, c.ws, false, c.st);
-  if (rc != TTT_OK) return rc;
+// Read of the nt tokens at Q (fused path), with the operand images of theta
+// already packed in the workspace.
+int launch_read_tokens(const Call& c, const uint16_t* Q, uint16_t* O, long long nt) {
+  Shape s = c.s;
+  s.n = nt;
+  s.tiles = static_cast<int>((nt + kTileM - 1) / kTileM);
   CUtensorMap tq;
   if (!make_token_map(&tq, Q, s)) return TTT_ECUDA;
   FwdParams fp;
@@ -602,8 +603,43 @@ int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) 
   fp.heads = s.H;
   fp.tiles = s.tiles;
   fp.status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
-  return launch_fwd<false>(s, tq, tq, fp, c.g.fwd, c.st);
+  const int grid = static_cast<int>(std::min<long long>(c.g.fwd, static_cast<long long>(s.H) * s.tiles));
+  return launch_fwd<false>(s, tq, tq, fp, grid, c.st);
 }
+
+int run_read(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
+  const Shape& s = c.s;
+  if (s.wide) return run_read_wide(c, Q, theta, O);
+  int rc = run_pack(s, theta, c.w, c.ws, false, c.st);
+  if (rc != TTT_OK) return rc;
+  return launch_read_tokens(c, Q, O, s.n);
+}
+
+// ------------------------------------------------------------------ host pipeline
+constexpr int kHostChunks = 8;           // most Q/O chunks of ttt_layer_host
+constexpr int kHostChunkMinTiles = 64;   // fewest 128-token tiles per chunk
+
+// Helper streams and events of one ttt_layer_host call, created per call and
+// destroyed once its work is enqueued (CUDA releases them when that work has
+// completed).
+struct HostPipe {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev[4 + 2 * kHostChunks] = {};
+  int n_ev = 0;
+  ~HostPipe() {
+    for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+    if (up) cudaStreamDestroy(up);
+    if (down) cudaStreamDestroy(down);
+  }
+  bool init(int events) {
+    if (cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    for (; n_ev < events; ++n_ev)
+      if (cudaEventCreateWithFlags(&ev[n_ev], cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+};
 
 // ------------------------------------------------------------------ fixed scratch
 // Scratch of ttt_read_noalloc.  In host code `g_noalloc_scratch` is only a
@@ -733,17 +769,76 @@ int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t*
   float* dw = reinterpret_cast<float*>(c.ws + c.w.convw);
   float* dth0 = reinterpret_cast<float*>(c.ws + c.w.th0);
   float* dthout = reinterpret_cast<float*>(c.ws + c.w.thout);
-  if (cudaMemcpyAsync(dq, Q_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
-      cudaMemcpyAsync(dk, K_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
-      cudaMemcpyAsync(dv, V_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
-      cudaMemcpyAsync(dw, conv_w_host, static_cast<size_t>(s.C) * 9 * 4, cudaMemcpyHostToDevice, c.st) !=
-          cudaSuccess ||
-      cudaMemcpyAsync(dth0, theta0_host, thb, cudaMemcpyHostToDevice, c.st) != cudaSuccess)
+  const size_t convb = static_cast<size_t>(s.C) * 9 * 4;
+  if (s.wide) {
+    // wide-head path: one copy each, in order on the caller's stream
+    if (cudaMemcpyAsync(dq, Q_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(dk, K_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(dv, V_host, tok, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(dw, conv_w_host, convb, cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(dth0, theta0_host, thb, cudaMemcpyHostToDevice, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    if ((rc = run_write(c, dims, dk, dv, dw, dth0, lr, steps, dthout)) != TTT_OK) return rc;
+    if ((rc = run_read(c, dq, dthout, dout)) != TTT_OK) return rc;
+    if (cudaMemcpyAsync(theta_out_host, dthout, thb, cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(O_host, dout, tok, cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    return TTT_OK;
+  }
+  // Fused path, pipelined over the two copy directions: the upload stream
+  // copies conv_w, theta0, V, K, then Q in chunks while the write runs; each
+  // chunk of Q is read as soon as it has landed, and its O goes back on the
+  // download stream while the next chunk is read.  Chunks are whole 128-token
+  // tiles, so each read launch covers exactly its own tokens.
+  const long long chunk_tiles =
+      std::max<long long>(kHostChunkMinTiles, (static_cast<long long>(s.tiles) + kHostChunks - 1) / kHostChunks);
+  const int chunks = static_cast<int>((s.tiles + chunk_tiles - 1) / chunk_tiles);
+  HostPipe hp;
+  if (!hp.init(4 + 2 * chunks)) return TTT_ECUDA;
+  cudaEvent_t ev_start = hp.ev[0], ev_kv = hp.ev[1], ev_th = hp.ev[2], ev_done = hp.ev[3];
+  cudaEvent_t* ev_q = hp.ev + 4;
+  cudaEvent_t* ev_o = hp.ev + 4 + chunks;
+  const size_t row_bytes = static_cast<size_t>(s.C) * 2;
+  auto chunk_rows = [&](int i, long long* t0) {
+    *t0 = i * chunk_tiles * kTileM;
+    return std::min<long long>(chunk_tiles * kTileM, s.n - *t0);
+  };
+  // everything earlier on the caller's stream comes first
+  if (cudaEventRecord(ev_start, c.st) != cudaSuccess || cudaStreamWaitEvent(hp.up, ev_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp.down, ev_start, 0) != cudaSuccess)
     return TTT_ECUDA;
+  if (cudaMemcpyAsync(dw, conv_w_host, convb, cudaMemcpyHostToDevice, hp.up) != cudaSuccess ||
+      cudaMemcpyAsync(dth0, theta0_host, thb, cudaMemcpyHostToDevice, hp.up) != cudaSuccess ||
+      cudaMemcpyAsync(dv, V_host, tok, cudaMemcpyHostToDevice, hp.up) != cudaSuccess ||
+      cudaMemcpyAsync(dk, K_host, tok, cudaMemcpyHostToDevice, hp.up) != cudaSuccess ||
+      cudaEventRecord(ev_kv, hp.up) != cudaSuccess)
+    return TTT_ECUDA;
+  for (int i = 0; i < chunks; ++i) {
+    long long t0;
+    const long long nt = chunk_rows(i, &t0);
+    if (cudaMemcpyAsync(dq + t0 * s.C, Q_host + t0 * s.C, nt * row_bytes, cudaMemcpyHostToDevice, hp.up) !=
+            cudaSuccess ||
+        cudaEventRecord(ev_q[i], hp.up) != cudaSuccess)
+      return TTT_ECUDA;
+  }
+  if (cudaStreamWaitEvent(c.st, ev_kv, 0) != cudaSuccess) return TTT_ECUDA;
   if ((rc = run_write(c, dims, dk, dv, dw, dth0, lr, steps, dthout)) != TTT_OK) return rc;
-  if ((rc = run_read(c, dq, dthout, dout)) != TTT_OK) return rc;
-  if (cudaMemcpyAsync(theta_out_host, dthout, thb, cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
-      cudaMemcpyAsync(O_host, dout, tok, cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
+  if ((rc = run_pack(s, dthout, c.w, c.ws, false, c.st)) != TTT_OK) return rc;
+  // theta* goes back once the write (and the pack that reads it) is done
+  if (cudaEventRecord(ev_th, c.st) != cudaSuccess || cudaStreamWaitEvent(hp.down, ev_th, 0) != cudaSuccess ||
+      cudaMemcpyAsync(theta_out_host, dthout, thb, cudaMemcpyDeviceToHost, hp.down) != cudaSuccess)
+    return TTT_ECUDA;
+  for (int i = 0; i < chunks; ++i) {
+    long long t0;
+    const long long nt = chunk_rows(i, &t0);
+    if (cudaStreamWaitEvent(c.st, ev_q[i], 0) != cudaSuccess) return TTT_ECUDA;
+    if ((rc = launch_read_tokens(c, dq + t0 * s.C, dout + t0 * s.C, nt)) != TTT_OK) return rc;
+    if (cudaEventRecord(ev_o[i], c.st) != cudaSuccess || cudaStreamWaitEvent(hp.down, ev_o[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(O_host + t0 * s.C, dout + t0 * s.C, nt * row_bytes, cudaMemcpyDeviceToHost, hp.down) !=
+            cudaSuccess)
+      return TTT_ECUDA;
+  }
+  if (cudaEventRecord(ev_done, hp.down) != cudaSuccess || cudaStreamWaitEvent(c.st, ev_done, 0) != cudaSuccess)
     return TTT_ECUDA;
   return TTT_OK;
 }
