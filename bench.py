@@ -8,9 +8,13 @@ and the read of Q.  Default workload: 1000 views x (37x37 + 5) tokens
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (under torchrun) every rank runs an independent replica of the
-workload (its own scene; the layer has no cross-scene exchange), so the
-scaling is weak and value = all ranks' tokens / max-over-ranks time.
+With N > 1 (under torchrun) the ranks run the write of ONE collection sharded
+by views: each rank holds 1000 views of an N x 1000-view collection,
+convolves and reads its own views, and per SGD step the ranks all-gather
+their gradient sums (NCCL, 3*heads*d*h floats each) and apply the same
+fixed-order update (test_layer_reconstruction_b200.sharded).  Per-GPU work is
+fixed, so the scaling is weak; value = all ranks' tokens / max-over-ranks
+time.  ``--replicas`` runs independent scenes instead (no exchange).
 ``--impl reference`` times the float64 CPU oracle on bounded samples of the
 same workload instead (rank 0 only).
 """
@@ -148,6 +152,13 @@ def replica_config(cfg, rank: int):
                            cfg.steps, cfg.lr, cfg.seed + 1000 * rank)
 
 
+def shard_views(cfg, rank: int, world: int):
+    """The collection of a sharded multi-GPU run (world x cfg.n_views views, the
+    workload's seed) and the contiguous views of `rank`."""
+    scene = cfg.with_views(cfg.n_views * world)
+    return scene, range(rank * cfg.n_views, (rank + 1) * cfg.n_views)
+
+
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time (all ranks call it, in the same order)."""
     import torch
@@ -213,7 +224,7 @@ def run_ours(args, cfg):
     import torch.distributed as dist
     from test_layer_reconstruction_b200 import build as tbuild
     from test_layer_reconstruction_b200 import inputs as tin
-    from test_layer_reconstruction_b200 import ttt
+    from test_layer_reconstruction_b200 import sharded, ttt
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -221,7 +232,8 @@ def run_ours(args, cfg):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
-    if world > 1:
+    distributed = world > 1 or (args.shard and "MASTER_ADDR" in os.environ)
+    if distributed:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     tbuild.build()
@@ -231,9 +243,13 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
-    # Each rank draws its own replica (seed offset by rank).
-    rcfg = replica_config(cfg, rank)
-    inp = tin.make_inputs(rcfg, device="cuda")
+    # N > 1: this rank's views of one collection (or, with --replicas, its own scene).
+    shard = (world > 1 and not args.replicas) or args.shard
+    if shard:
+        scene, views = shard_views(cfg, rank, world)
+        inp = tin.make_inputs(scene, device="cuda", views=views)
+    else:
+        inp = tin.make_inputs(replica_config(cfg, rank), device="cuda")
     Q = inp["Q"].to(torch.bfloat16).contiguous()
     K = inp["K"].to(torch.bfloat16).contiguous()
     V = inp["V"].to(torch.bfloat16).contiguous()
@@ -244,9 +260,23 @@ def run_ours(args, cfg):
     theta = torch.empty_like(theta0)
     O = torch.empty_like(Q)
     ws = ttt.make_workspace(cfg, ttt.OP_LAYER)
+    if shard:
+        n_total = cfg.n * world
+        gather = sharded.all_gather_rows() if distributed else (lambda t: t.reshape(1, -1))
+        ops = sharded.ShardOps(
+            conv=lambda V_, w_, dm: ttt.shortconv2d(V_, w_, dm),
+            grad=lambda K_, Vp_, th_, dm: ttt.grad(K_, Vp_, th_, dm, workspace=ws),
+            update=lambda th_, g_, sc_, dm: ttt.sgd_update(th_, g_, sc_, dm),
+            read=lambda Q_, th_, dm: ttt.read(Q_, th_, dm, O=O, workspace=ws))
+
+        def layer_call(Q_, K_, V_, w_, th0_):
+            return sharded.layer_sharded(Q_, K_, V_, w_, th0_, cfg.lr, cfg.steps, cfg, n_total, gather, ops)
+    else:
+        def layer_call(Q_, K_, V_, w_, th0_):
+            return ttt.layer(Q_, K_, V_, w_, th0_, cfg.lr, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
 
     def step():
-        ttt.layer(Q, K, V, conv_w, theta0, cfg.lr, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
+        layer_call(Q, K, V, conv_w, theta0)
 
     for _ in range(args.warmup):
         step()
@@ -307,7 +337,40 @@ def run_ours(args, cfg):
 
     # end to end through the host-buffer entry point
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and shard:
+        # the sharded layer from pinned host buffers: this rank's inputs up, O and theta* back
+        hq, hk, hv = (t.cpu().pin_memory() for t in (Q, K, V))
+        hw = conv_w.cpu().pin_memory()
+        ht0 = theta0.cpu().pin_memory()
+        hth = torch.empty_like(ht0).pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        h2d = 3 * hq.numel() * 2 + hw.numel() * 4 + ht0.numel() * 4
+        d2h = ho.numel() * 2 + hth.numel() * 4
+        dq, dk, dv, dw, dt = (torch.empty_like(t) for t in (Q, K, V, conv_w, theta0))
+
+        def host_call():
+            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (dw, hw), (dt, ht0)):
+                dst.copy_(src, non_blocking=True)
+            th_, O_ = layer_call(dq, dk, dv, dw, dt)
+            hth.copy_(th_, non_blocking=True)
+            ho.copy_(O_, non_blocking=True)
+
+        host_call()
+        torch.cuda.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            host_call()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = f0.elapsed_time(f1) / args.e2e_steps
+        e_max = max_over_ranks(e_ms, world, "cuda")
+        e2e = {"value": whole_job_tokens_per_s(world, cfg.n, e_max), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "wall_s_per_step": (time.perf_counter() - t0) / args.e2e_steps}
+    elif args.e2e_steps > 0:
         ws_h = ttt.make_workspace(cfg, ttt.OP_LAYER_HOST)
         hq, hk, hv = (t.cpu().pin_memory() for t in (Q, K, V))
         hw = conv_w.cpu().pin_memory()
@@ -395,12 +458,14 @@ def run_ours(args, cfg):
             "config": {"workload": cfg.name, "n_views": cfg.n_views, "tokens": cfg.n, "heads": cfg.heads,
                        "d": cfg.d, "h": cfg.h, "steps": cfg.steps, "lr": cfg.lr,
                        "l2": f"no flush: every token tensor ({cfg.n * cfg.heads * cfg.d * 2 / 1e9:.2f} GB) exceeds the 126 MB L2",
-                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+                       "parallelism": (f"{world} GPUs: one {cfg.n_views * world}-view collection sharded by views "
+                                       f"({cfg.n_views} per GPU), gradient all-gather per step (NCCL)" if shard
+                                       else f"{world} independent replicas" if world > 1 else "1 GPU")},
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": gpu_launches, "clocks": clk, "sweep": sweep, "paths": paths,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if distributed:
         dist.destroy_process_group()
     return 0
 
@@ -446,6 +511,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the view-count sweep and write/read split")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1: independent scenes per GPU instead of one collection sharded by views")
+    ap.add_argument("--shard", action="store_true",
+                    help="run the view-sharded layer even on one GPU (under torchrun: with the NCCL all-gather)")
     args = ap.parse_args()
     from test_layer_reconstruction_b200 import inputs as tin
     cfg = tin.CONFIGS[args.config]

@@ -104,6 +104,35 @@ int ttt_write(const ttt_dims* dims, const uint16_t* K, const uint16_t* V,
               const float* conv_w, const float* theta0, float lr, int steps,
               float* theta_out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* The write sharded over processes (one collection's views split between
+ * ranks).  The loss gradient is a sum of per-token terms (VGG-T^3: Offline
+ * Feed-Forward 3D Reconstruction at Scale, Sec. 3.4, Eq. 5), so a rank
+ * evaluates it on its own views, the ranks exchange these sums, and every
+ * rank applies the same step.  Per rank: V' = ttt_shortconv2d(V) of its views
+ * once, then per step
+ *   ttt_grad on (K, V') of its views -> its gradient sum,
+ *   an all-gather of the ranks' sums (by the caller, e.g. NCCL),
+ *   ttt_sgd_update with all of them and scale = lr * 2 / n_total.
+ * With one rank this is ttt_write. */
+
+/* grad = d/dtheta of (1/2) sum_i ||T_theta(k_i) - vp_i||^2 over the n tokens
+ * that dims describe (the gradient of Eq. 3's loss is (2/n_total) times the
+ * sum of the ranks' grads).  K, Vp: bf16 [n][heads][d], Vp = ShortConv2D(V)
+ * of the same views; theta, grad: f32, theta's packed layout.  FP32
+ * accumulation over bf16 operands, summed in a fixed order (deterministic).
+ * Workspace: ttt_workspace_bytes(dims, TTT_OP_WRITE). */
+int ttt_grad(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const float* theta,
+             float* grad, void* workspace, size_t workspace_bytes, void* stream);
+
+/* theta_out = theta_in - scale * (grads[0] + ... + grads[n_grads - 1]) for
+ * every element, the sum taken in index order, so every rank that applies
+ * the same inputs gets the same bits.  grads: n_grads >= 1 contiguous f32
+ * buffers of theta's size (for example an all-gather of the ranks' ttt_grad
+ * outputs in rank order).  Only heads, d and h of dims are used.  theta_out
+ * may alias theta_in.  Needs no workspace. */
+int ttt_sgd_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads,
+                   float scale, float* theta_out, void* stream);
+
 /* Read (Eq. 4): O = T_theta(Q) with frozen theta (query mode).  dims describe
  * Q's token count through n_views/grid/n_special; only n, heads, d, h are used. */
 int ttt_read(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O,

@@ -435,9 +435,48 @@ int wide_forward_chunk(const Call& c, cublasHandle_t hd, const uint16_t* X, int 
   return launch_status();
 }
 
-// The write of the wide path: per step, per head, per token chunk
+// dW of one head of the wide path over all tokens, per token chunk
 //   Z1, Z3, A (forward) -> E = A W2 - V' -> dA = E W2^T -> dZ1, dZ3
 //   -> dW1 += K^T dZ1, dW3 += K^T dZ3, dW2 += A^T E   (FP32, Eq. 5)
+// into the workspace accumulator; the operand image of theta is current.
+int wide_grad_head(const Call& c, cublasHandle_t hd, const uint16_t* K, const uint16_t* vp, int head) {
+  const Shape& s = c.s;
+  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
+  float* acc = reinterpret_cast<float*>(c.ws + c.w.acc);
+  uint8_t* eb = c.ws + c.w.eb;
+  const int ldx = s.H * s.D;
+  const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;   // [h][D]
+  int rc;
+  for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
+    const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
+    const float beta = t0 == 0 ? 0.f : 1.f;
+    if ((rc = wide_forward_chunk(c, hd, K, head, t0, nc)) != TTT_OK) return rc;
+    // E = A W2 - V' (the chunk's V' rows first copied into E)
+    if (cudaMemcpy2DAsync(eb, static_cast<size_t>(s.D) * 2, vp + (static_cast<size_t>(t0) * s.H + head) * s.D,
+                          static_cast<size_t>(ldx) * 2, static_cast<size_t>(s.D) * 2, nc, cudaMemcpyDeviceToDevice,
+                          c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    if (!gemm_rm(hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, -1.f, eb, CUDA_R_16BF, s.D) ||
+        !gemm_rm(hd, false, true, nc, s.h, s.D, 1.f, eb, s.D, w2, s.D, 0.f, c.ws + c.w.da, CUDA_R_16BF, s.h))
+      return TTT_ECUDA;
+    const long long n8 = static_cast<long long>(nc) * s.h / 8;
+    wide_dz_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<uint4*>(c.ws + c.w.z1),
+                                                           reinterpret_cast<uint4*>(c.ws + c.w.z3),
+                                                           reinterpret_cast<const uint4*>(c.ws + c.w.da), n8);
+    if ((rc = launch_status()) != TTT_OK) return rc;
+    const uint16_t* kc = K + (static_cast<size_t>(t0) * s.H + head) * s.D;
+    if (!gemm_rm(hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z1, s.h, beta, acc, CUDA_R_32F, s.h) ||
+        !gemm_rm(hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z3, s.h, beta, acc + per, CUDA_R_32F,
+                 s.h) ||
+        !gemm_rm(hd, true, false, s.h, s.D, nc, 1.f, c.ws + c.w.ab, s.h, eb, s.D, beta, acc + 2 * per, CUDA_R_32F,
+                 s.D))
+      return TTT_ECUDA;
+  }
+  return TTT_OK;
+}
+
+// The write of the wide path: per step and head, dW over all token chunks,
 // then theta_out = theta_in - lr (2/n) dW for the head.
 int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
                    const float* theta0, float lr, int steps, float* theta_out) {
@@ -454,47 +493,35 @@ int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const u
   WideCall wc(c);
   if (!wc.ok) return TTT_ECUDA;
   const size_t per = static_cast<size_t>(s.D) * s.h;
-  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
-  float* acc = reinterpret_cast<float*>(c.ws + c.w.acc);
-  uint8_t* eb = c.ws + c.w.eb;
-  const int ldx = s.H * s.D;
+  const float* acc = reinterpret_cast<const float*>(c.ws + c.w.acc);
   const float scale = lr * 2.0f / static_cast<float>(s.n);
   for (int step = 0; step < steps; ++step) {
     const float* th_in = step == 0 ? theta0 : theta_out;
     if ((rc = wide_cast(c, th_in)) != TTT_OK) return rc;
     for (int head = 0; head < s.H; ++head) {
-      const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;   // [h][D]
-      for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
-        const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
-        const float beta = t0 == 0 ? 0.f : 1.f;
-        if ((rc = wide_forward_chunk(c, wc.hd, K, head, t0, nc)) != TTT_OK) return rc;
-        // E = A W2 - V' (the chunk's V' rows first copied into E)
-        if (cudaMemcpy2DAsync(eb, static_cast<size_t>(s.D) * 2, vp + (static_cast<size_t>(t0) * s.H + head) * s.D,
-                              static_cast<size_t>(ldx) * 2, static_cast<size_t>(s.D) * 2, nc,
-                              cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
-          return TTT_ECUDA;
-        if (!gemm_rm(wc.hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, -1.f, eb, CUDA_R_16BF,
-                     s.D) ||
-            !gemm_rm(wc.hd, false, true, nc, s.h, s.D, 1.f, eb, s.D, w2, s.D, 0.f, c.ws + c.w.da, CUDA_R_16BF, s.h))
-          return TTT_ECUDA;
-        const long long n8 = static_cast<long long>(nc) * s.h / 8;
-        wide_dz_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<uint4*>(c.ws + c.w.z1),
-                                                               reinterpret_cast<uint4*>(c.ws + c.w.z3),
-                                                               reinterpret_cast<const uint4*>(c.ws + c.w.da), n8);
-        if ((rc = launch_status()) != TTT_OK) return rc;
-        const uint16_t* kc = K + (static_cast<size_t>(t0) * s.H + head) * s.D;
-        if (!gemm_rm(wc.hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z1, s.h, beta, acc, CUDA_R_32F,
-                     s.h) ||
-            !gemm_rm(wc.hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z3, s.h, beta, acc + per,
-                     CUDA_R_32F, s.h) ||
-            !gemm_rm(wc.hd, true, false, s.h, s.D, nc, 1.f, c.ws + c.w.ab, s.h, eb, s.D, beta, acc + 2 * per,
-                     CUDA_R_32F, s.D))
-          return TTT_ECUDA;
-      }
+      if ((rc = wide_grad_head(c, wc.hd, K, vp, head)) != TTT_OK) return rc;
       wide_sgd_kernel<<<elementwise_grid(static_cast<long long>(3 * per) / 8), 256, 0, c.st>>>(
           th_in, theta_out, acc, s.H, s.D, s.h, head, scale);
       if ((rc = launch_status()) != TTT_OK) return rc;
     }
+  }
+  return TTT_OK;
+}
+
+// The gradient (1/2) d/dtheta sum_i ||T(k_i) - v'_i||^2 of the wide path.
+int run_grad_wide(const Call& c, const uint16_t* K, const uint16_t* vp, const float* theta, float* grad) {
+  const Shape& s = c.s;
+  WideCall wc(c);
+  if (!wc.ok) return TTT_ECUDA;
+  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const float* acc = reinterpret_cast<const float*>(c.ws + c.w.acc);
+  int rc = wide_cast(c, theta);
+  if (rc != TTT_OK) return rc;
+  for (int head = 0; head < s.H; ++head) {
+    if ((rc = wide_grad_head(c, wc.hd, K, vp, head)) != TTT_OK) return rc;
+    wide_grad_kernel<<<elementwise_grid(static_cast<long long>(3 * per) / 8), 256, 0, c.st>>>(grad, acc, s.H, s.D,
+                                                                                              s.h, head);
+    if ((rc = launch_status()) != TTT_OK) return rc;
   }
   return TTT_OK;
 }
@@ -523,26 +550,24 @@ int run_read_wide(const Call& c, const uint16_t* Q, const float* theta, uint16_t
   return TTT_OK;
 }
 
-int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
-              const float* theta0, float lr, int steps, float* theta_out) {
+// One gradient pass of the fused path over (K, V'): operand images of theta,
+// forward (E = T(K) - V'), backward partials, and the fixed-order reduction.
+struct GradPass {
+  CUtensorMap tk, tvp, tku, teu;
+  FwdParams fp;
+  BwdParams bp;
+  UpdateParams up;
+  long long red_threads;
+};
+
+bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradPass* gp) {
   const Shape& s = c.s;
-  if (s.wide) return run_write_wide(c, dm, K, V, conv_w, theta0, lr, steps, theta_out);
-  uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
   uint16_t* e = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
   unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
-  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
-  if (rc != TTT_OK) return rc;
-  if (steps == 0) {
-    if (theta_out != theta0 &&
-        cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
-      return TTT_ECUDA;
-    return TTT_OK;
-  }
-  CUtensorMap tk, tvp, tku, teu;
-  if (!make_token_map(&tk, K, s) || !make_token_map(&tvp, vp, s) || !make_token_map(&tku, K, s, kUnit) ||
-      !make_token_map(&teu, e, s, kUnit))
-    return TTT_ECUDA;
-  FwdParams fp;
+  if (!make_token_map(&gp->tk, K, s) || !make_token_map(&gp->tvp, vp, s) || !make_token_map(&gp->tku, K, s, kUnit) ||
+      !make_token_map(&gp->teu, e, s, kUnit))
+    return false;
+  FwdParams& fp = gp->fp;
   fp.w13_img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.w13);
   fp.w2_img = reinterpret_cast<const __half*>(c.ws + c.w.w2h);
   fp.out = reinterpret_cast<__nv_bfloat16*>(e);
@@ -550,7 +575,7 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   fp.heads = s.H;
   fp.tiles = s.tiles;
   fp.status = status;
-  BwdParams bp;
+  BwdParams& bp = gp->bp;
   bp.wt_img = reinterpret_cast<const uint32_t*>(c.ws + c.w.wt);
   bp.partials = reinterpret_cast<float*>(c.ws + c.w.part);
   bp.n = fp.n;
@@ -559,9 +584,8 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   bp.slices = s.slices;
   bp.max_contrib = c.g.max_contrib;
   bp.status = status;
-  UpdateParams up;
+  UpdateParams& up = gp->up;
   up.partials = bp.partials;
-  up.theta_out = theta_out;
   up.heads = s.H;
   up.d = s.D;
   up.h = s.h;
@@ -570,21 +594,56 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   up.max_contrib = c.g.max_contrib;
   up.n_items = static_cast<long long>(s.H) * s.units;
   up.grid = c.g.bwd_groups;
-  up.scale = lr * 2.0f / static_cast<float>(s.n);
-  const long long red_threads = static_cast<long long>(s.H) * s.slices * 3 * 128 * s.D;
+  gp->red_threads = static_cast<long long>(s.H) * s.slices * 3 * 128 * s.D;
+  return true;
+}
+
+// With theta_in: out = theta_in - scale * g (one SGD step).  Without: out = g.
+int run_grad_pass(const Call& c, GradPass& gp, const float* theta, const float* theta_in, float scale, float* out) {
+  const Shape& s = c.s;
+  int rc;
+  if ((rc = run_pack(s, theta, c.w, c.ws, true, c.st)) != TTT_OK) return rc;
+  if ((rc = launch_fwd<true>(s, gp.tk, gp.tvp, gp.fp, c.g.fwd, c.st)) != TTT_OK) return rc;
+  if ((rc = launch_bwd(s, gp.tku, gp.teu, gp.bp, c.g.bwd, c.st)) != TTT_OK) return rc;
+  gp.up.theta_in = theta_in;
+  gp.up.theta_out = out;
+  gp.up.scale = scale;
+  {
+    ProfScope prof(KK_REDUCE, c.st);
+    reduce_sgd_kernel<<<static_cast<unsigned>((gp.red_threads + 255) / 256), 256, 0, c.st>>>(gp.up);
+  }
+  return launch_status();
+}
+
+int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
+              const float* theta0, float lr, int steps, float* theta_out) {
+  const Shape& s = c.s;
+  if (s.wide) return run_write_wide(c, dm, K, V, conv_w, theta0, lr, steps, theta_out);
+  uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
+  if (rc != TTT_OK) return rc;
+  if (steps == 0) {
+    if (theta_out != theta0 &&
+        cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    return TTT_OK;
+  }
+  GradPass gp;
+  if (!setup_grad_pass(c, K, vp, &gp)) return TTT_ECUDA;
+  const float scale = lr * 2.0f / static_cast<float>(s.n);
   for (int step = 0; step < steps; ++step) {
     const float* th_in = step == 0 ? theta0 : theta_out;
-    if ((rc = run_pack(s, th_in, c.w, c.ws, true, c.st)) != TTT_OK) return rc;
-    if ((rc = launch_fwd<true>(s, tk, tvp, fp, c.g.fwd, c.st)) != TTT_OK) return rc;
-    if ((rc = launch_bwd(s, tku, teu, bp, c.g.bwd, c.st)) != TTT_OK) return rc;
-    up.theta_in = th_in;
-    {
-      ProfScope prof(KK_REDUCE, c.st);
-      reduce_sgd_kernel<<<static_cast<unsigned>((red_threads + 255) / 256), 256, 0, c.st>>>(up);
-    }
-    if ((rc = launch_status()) != TTT_OK) return rc;
+    if ((rc = run_grad_pass(c, gp, th_in, th_in, scale, theta_out)) != TTT_OK) return rc;
   }
   return TTT_OK;
+}
+
+// The gradient of (1/2) sum_i ||T(k_i) - v'_i||^2 over the call's tokens.
+int run_grad(const Call& c, const uint16_t* K, const uint16_t* vp, const float* theta, float* grad) {
+  if (c.s.wide) return run_grad_wide(c, K, vp, theta, grad);
+  GradPass gp;
+  if (!setup_grad_pass(c, K, vp, &gp)) return TTT_ECUDA;
+  return run_grad_pass(c, gp, theta, nullptr, 1.f, grad);
 }
 
 // Read of the nt tokens at Q (fused path), with the operand images of theta
@@ -725,6 +784,32 @@ int ttt_write(const ttt_dims* dims, const uint16_t* K, const uint16_t* V, const 
   int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
   return run_write(c, dims, K, V, conv_w, theta0, lr, steps, theta_out);
+}
+
+int ttt_grad(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const float* theta, float* grad,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!K || !Vp || !theta || !grad) return TTT_EINVAL;
+  if (!aligned(K) || !aligned(Vp) || !aligned(theta) || !aligned(grad)) return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  return run_grad(c, K, Vp, theta, grad);
+}
+
+int ttt_sgd_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads, float scale,
+                   float* theta_out, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != TTT_OK) return rc;
+  if (!theta_in || !grads || !theta_out || n_grads < 1) return TTT_EINVAL;
+  if (!aligned(theta_in) || !aligned(grads) || !aligned(theta_out)) return TTT_EALIGN;
+  const long long count = 3LL * s.H * s.D * s.h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    ProfScope prof(KK_REDUCE, st);
+    sgd_sum_kernel<<<elementwise_grid(count), 256, 0, st>>>(theta_in, grads, n_grads, count, scale, theta_out);
+  }
+  return launch_status();
 }
 
 int ttt_read(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O, void* workspace,

@@ -7,7 +7,13 @@
 //   theta_out = theta_in - lr * (2/n) * g
 // (plain SGD on the mean-squared loss; the 2/n of its gradient is applied
 // here).  theta_out may alias theta_in: each element is read and written by
-// one thread.
+// one thread.  With theta_in null the kernel writes g itself (the gradient of
+// (1/2) sum_i ||T(k_i) - v'_i||^2 over the call's tokens) into theta_out, for
+// a write whose tokens are sharded over several processes.
+//
+// sgd_sum: theta_out = theta_in - scale * (g_0 + g_1 + ... + g_{r-1}) over r
+// gathered gradients, summed in index order for every element, so every
+// process that applies it gets the same bits.
 //
 // pack_images: theta (f32) -> round-to-nearest-even operand images, hidden
 // units padded with zeros up to HIDP:
@@ -26,7 +32,7 @@ namespace ttt {
 
 struct UpdateParams {
   const float* partials;
-  const float* theta_in;
+  const float* theta_in;   // null: write the gradient itself
   float* theta_out;
   int heads, d, h, slices, units, max_contrib;
   long long n_items;   // heads * units
@@ -60,7 +66,21 @@ __global__ void reduce_sgd_kernel(const UpdateParams p) {
   else if (m == 1) off = hdh + static_cast<size_t>(head) * D * p.h + static_cast<size_t>(i) * p.h + hid;
   else off = 2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(hid) * D + i;
   // the backward kernel accumulates 2 dW1^T (its chain rule runs on z1/2): halve it, exactly
-  p.theta_out[off] = p.theta_in[off] - (m == 0 ? 0.5f * p.scale : p.scale) * g;
+  if (p.theta_in)
+    p.theta_out[off] = p.theta_in[off] - (m == 0 ? 0.5f * p.scale : p.scale) * g;
+  else
+    p.theta_out[off] = m == 0 ? 0.5f * g : g;
+}
+
+// theta_out = theta_in - scale * sum_r grads[r * count + e], r in order.
+__global__ void sgd_sum_kernel(const float* theta_in, const float* __restrict__ grads, int n_grads,
+                               long long count, float scale, float* theta_out) {
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float g = grads[e];
+    for (int r = 1; r < n_grads; ++r) g += grads[static_cast<long long>(r) * count + e];
+    theta_out[e] = theta_in[e] - scale * g;
+  }
 }
 
 struct PackParams {

@@ -13,6 +13,7 @@
 //   wide_dz_kernel    dZ1 = dA Z3 s (1 + Z1 (1 - s)), dZ3 = dA Z1 s, s = sigmoid(Z1)
 //   wide_cast_kernel  bf16 copy of theta (same layout) for the GEMM operands
 //   wide_sgd_kernel   theta_out = theta_in - scale * dW of one head
+//   wide_grad_kernel  dW of one head into a gradient in theta's layout
 // All elementwise math is FP32 on bf16 storage, 8 elements (16 bytes) per
 // thread and iteration; these steps are HBM-bound.
 #pragma once
@@ -91,6 +92,16 @@ __global__ void wide_sgd_kernel(const float* theta_in, float* theta_out, const f
     const long long m = e / per, r = e % per;
     const long long off = m * heads * per + static_cast<long long>(head) * per + r;
     theta_out[off] = theta_in[off] - scale * dw[e];
+  }
+}
+
+// grad = dW of head `head`, scattered into theta's per-head layout.
+__global__ void wide_grad_kernel(float* grad, const float* __restrict__ dw, int heads, int d, int h, int head) {
+  const long long per = static_cast<long long>(d) * h;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < 3 * per;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long m = e / per, r = e % per;
+    grad[m * heads * per + static_cast<long long>(head) * per + r] = dw[e];
   }
 }
 

@@ -16,14 +16,14 @@ from .inputs import LayerConfig
 
 __all__ = [
     "TTTError", "Dims", "library_path", "load_library", "workspace_bytes", "make_workspace",
-    "shortconv2d", "write", "read", "layer", "layer_host", "check_status",
+    "shortconv2d", "write", "grad", "sgd_update", "read", "layer", "layer_host", "check_status",
     "OP_WRITE", "OP_READ", "OP_LAYER", "OP_LAYER_HOST", "EXPORTED_SYMBOLS", "profile_start", "profile_stop",
 ]
 
 OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
 EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
                     "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
-                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc")
+                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_grad", "ttt_sgd_update")
 KERNEL_KINDS = 6
 
 
@@ -80,6 +80,8 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_shortconv2d.argtypes = [DP, P, P, P, P]
     lib.ttt_write.argtypes = [DP, P, P, P, P, F, I, P, P, S, P]
     lib.ttt_read.argtypes = [DP, P, P, P, P, S, P]
+    lib.ttt_grad.argtypes = [DP, P, P, P, P, P, S, P]
+    lib.ttt_sgd_update.argtypes = [DP, P, P, I, F, P, P]
     lib.ttt_layer.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
     lib.ttt_layer_host.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
     lib.ttt_check_status.argtypes = [P, P]
@@ -92,7 +94,7 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_kernel_name.argtypes = [I]
     lib.ttt_kernel_name.restype = ctypes.c_char_p
     for f in ("ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer", "ttt_layer_host", "ttt_check_status",
-              "ttt_profile_start", "ttt_profile_stop"):
+              "ttt_profile_start", "ttt_profile_stop", "ttt_grad", "ttt_sgd_update"):
         getattr(lib, f).restype = I
     _LIB = lib
     return lib
@@ -154,6 +156,30 @@ def write(K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, wor
                                     _dev(conv_w, torch.float32, "conv_w"), _dev(theta0, torch.float32, "theta0"),
                                     float(lr), int(steps), _dev(theta_out, torch.float32, "theta_out"),
                                     ws.data_ptr(), ws.numel(), _stream()), "ttt_write")
+    return theta_out
+
+
+def grad(K, Vp, theta, dims, out=None, workspace=None) -> torch.Tensor:
+    """d/dtheta of (1/2) sum_i ||T_theta(k_i) - v'_i||^2 over the tokens of (K, Vp) (Eq. 5 summand sum)."""
+    dm = Dims.of(dims)
+    out = torch.empty_like(theta) if out is None else out
+    ws = make_workspace(dm, OP_WRITE, K.device) if workspace is None else workspace
+    _check(load_library().ttt_grad(ctypes.byref(dm), _dev(K, torch.bfloat16, "K"), _dev(Vp, torch.bfloat16, "Vp"),
+                                   _dev(theta, torch.float32, "theta"), _dev(out, torch.float32, "grad"),
+                                   ws.data_ptr(), ws.numel(), _stream()), "ttt_grad")
+    return out
+
+
+def sgd_update(theta_in, grads, scale: float, dims, theta_out=None) -> torch.Tensor:
+    """theta_out = theta_in - scale * sum_r grads[r] (rows of `grads` summed in order); returns theta_out."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta_in) if theta_out is None else theta_out
+    if grads.numel() % theta_in.numel() != 0:
+        raise ValueError("grads must hold whole gradients of theta's size")
+    n_grads = grads.numel() // theta_in.numel()
+    _check(load_library().ttt_sgd_update(ctypes.byref(dm), _dev(theta_in, torch.float32, "theta_in"),
+                                         _dev(grads, torch.float32, "grads"), int(n_grads), float(scale),
+                                         _dev(theta_out, torch.float32, "theta_out"), _stream()), "ttt_sgd_update")
     return theta_out
 
 

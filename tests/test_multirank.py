@@ -1,11 +1,12 @@
-"""The N > 1 path of bench.py on CPU: two gloo ranks, each an independent
-replica of the workload (the layer has no cross-scene exchange, so there is no
-data-path collective).
+"""The N > 1 pieces of bench.py on CPU, on two gloo ranks: the views each rank
+holds in a sharded run (one collection, contiguous halves), the independent
+replicas of ``--replicas``, the max-over-ranks step time, and the reference
+arm.  The sharded write itself is tested in tests/test_multirank_sharded.py.
 
-Checks the pieces the multi-GPU run is made of: each rank draws its own scene,
-the step time is the slowest rank's (an all-reduce MAX that every rank calls),
-value = all ranks' tokens over that time, and the reference arm runs on rank 0
-alone while the other ranks exit 0 without work.
+Checked: with ``--replicas`` each rank draws its own scene; the step time is
+the slowest rank's (an all-reduce MAX that every rank calls); value = all
+ranks' tokens over that time; the reference arm runs on rank 0 alone while
+the other ranks exit 0 without work.
 """
 import contextlib
 import datetime
@@ -38,6 +39,7 @@ def _worker(rank: int, world: int, port: int, q) -> None:
         ms = [3.0, 5.0][rank]
         ms_max = bench.max_over_ranks(ms, world, "cpu")
         rcfg = bench.replica_config(TINY, rank)
+        scene, views = bench.shard_views(TINY, rank, world)
         k = tin.make_inputs(rcfg)["K"]
         mine = torch.tensor([float(k.double().sum())], dtype=torch.float64)
         sums = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
@@ -47,7 +49,7 @@ def _worker(rank: int, world: int, port: int, q) -> None:
         with contextlib.redirect_stdout(out):
             ret = bench.run_reference(args, TINY)
         q.put((rank, ms_max, bench.whole_job_tokens_per_s(world, TINY.n, ms_max), rcfg.seed,
-               [float(t) for t in sums], ret, out.getvalue()))
+               [float(t) for t in sums], ret, out.getvalue(), (scene.n_views, scene.seed, list(views))))
     finally:
         dist.destroy_process_group()
 
@@ -63,7 +65,10 @@ def test_two_gloo_ranks_replicas_timing_and_reference_arm():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, max0, val0, seed0, sums0, ret0, out0), (r1, max1, val1, seed1, sums1, ret1, out1) = results
+    (r0, max0, val0, seed0, sums0, ret0, out0, sv0), (r1, max1, val1, seed1, sums1, ret1, out1, sv1) = results
+    # sharded runs: one collection of 2 x n_views views (the workload's seed), contiguous halves
+    assert sv0 == (2 * TINY.n_views, TINY.seed, list(range(TINY.n_views)))
+    assert sv1 == (2 * TINY.n_views, TINY.seed, list(range(TINY.n_views, 2 * TINY.n_views)))
     assert (r0, r1) == (0, 1)
     # the slowest rank's time, on every rank
     assert max0 == max1 == 5.0
