@@ -32,6 +32,20 @@ Readings taken where the pages are silent or disagree:
   bias, depthwise over all heads*d channels, weights shared by all views.
 * Special tokens are the first ``n_special`` tokens of each view.
 
+The pages' own inner loop (dot-product loss and Muon; a later step of the
+build, pinned here before any kernel) takes these readings:
+
+* Dot-product loss ([summary] Sec. 3.4, "The dot product loss": the per-token
+  loss is T(k)^T v, and the arg-min form implies a minus sign):
+  L = -(1/n) sum_i <T(k_i), v'_i>, on V' as for the mean-squared loss.  The
+  1/n is immaterial under Muon, whose step is scale-invariant.
+* Muon ("TTT MLP Architecture and Inner Optimization": 5 Newton-Schulz
+  iterations, learning rate 0.1; the pages give no polynomial, momentum or
+  shape factor): per weight matrix of a head, X_0 = G / ||G||_F and the cubic
+  Newton-Schulz iteration for the orthogonal polar factor,
+  X <- 1.5 X - 0.5 X X^T X, five times; then theta <- theta - lr * X_5.  No
+  momentum (one or two steps), no shape factor.
+
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against
 facts that do not come from this file (library routines, finite differences,
 closed forms, brute force, invariants).
@@ -46,6 +60,7 @@ import numpy as np
 __all__ = [
     "Dims", "shortconv2d", "sigmoid", "swiglu_forward", "mse_loss", "mse_grad", "mse_grad_chunked",
     "sgd_write", "read", "layer", "LinearModel", "SwiGLUModel", "ChunkedSwiGLUModel",
+    "dot_loss", "dot_grad", "newton_schulz", "muon_write", "DotSwiGLUModel", "DotLinearModel",
 ]
 
 
@@ -216,6 +231,95 @@ def sgd_write(K, Vp, theta0: Sequence[np.ndarray], lr: float, steps: int,
         losses.append(mse_loss(model.forward(K, theta), Vp))
         g = model.grad(K, Vp, theta)
         theta = [w - lr * gw for w, gw in zip(theta, g)]
+    return theta, losses
+
+
+# ---------------------------------------------------------------------------
+# The pages' own inner loop: dot-product loss and Muon ([summary] Sec. 3.4,
+# "The dot product loss"; "TTT MLP Architecture and Inner Optimization")
+# ---------------------------------------------------------------------------
+
+def dot_loss(Y: np.ndarray, Vp: np.ndarray) -> float:
+    """-(1/n) * sum_i <y_i, v'_i> over all n tokens."""
+    n = Y.shape[0]
+    return float(-np.sum(Y * Vp) / n)
+
+
+def dot_grad(K, Vp, W1, W3, W2) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradient of dot_loss(T(K), V') with respect to (W1, W3, W2).
+
+    The chain rule of mse_grad with dL/dY = G = -V'/n (the loss is linear in
+    Y, so G does not depend on theta):
+      dW2 = A^T G,  dA = G W2^T,  dZ1 = dA * Z3 * S * (1 + Z1 (1 - S)),
+      dZ3 = dA * Z1 * S,  dW1 = K^T dZ1,  dW3 = K^T dZ3.
+    """
+    n = K.shape[0]
+    _, Z1, Z3, A = swiglu_forward(K, W1, W3, W2)
+    S = sigmoid(Z1)
+    G = -Vp / n
+    dW2 = A.T @ G
+    dA = G @ W2.T
+    dZ1 = dA * Z3 * S * (1.0 + Z1 * (1.0 - S))
+    dZ3 = dA * Z1 * S
+    return K.T @ dZ1, K.T @ dZ3, dW2
+
+
+def newton_schulz(G: np.ndarray, iters: int = 5) -> np.ndarray:
+    """Muon's orthogonalised update of one matrix: X_0 = G / ||G||_F, then
+    X <- 1.5 X - 0.5 X X^T X, ``iters`` times (zero for G = 0)."""
+    G = np.asarray(G, np.float64)
+    nrm = np.sqrt(np.sum(G * G))
+    if nrm == 0.0:
+        return np.zeros_like(G)
+    X = G / nrm
+    for _ in range(iters):
+        X = 1.5 * X - 0.5 * (X @ X.T) @ X
+    return X
+
+
+class DotSwiGLUModel:
+    """SwiGLU fast weights under the dot-product loss."""
+
+    @staticmethod
+    def forward(X, theta):
+        return swiglu_forward(X, *theta)[0]
+
+    @staticmethod
+    def loss(Y, Vp):
+        return dot_loss(Y, Vp)
+
+    @staticmethod
+    def grad(X, Vp, theta):
+        return dot_grad(X, Vp, *theta)
+
+
+class DotLinearModel:
+    """T(x) = x W under the dot-product loss, used only to pin the Muon loop
+    against a closed form."""
+
+    @staticmethod
+    def forward(X, theta):
+        return X @ theta[0]
+
+    @staticmethod
+    def loss(Y, Vp):
+        return dot_loss(Y, Vp)
+
+    @staticmethod
+    def grad(X, Vp, theta):
+        return (-(X.T @ Vp) / X.shape[0],)
+
+
+def muon_write(K, Vp, theta0: Sequence[np.ndarray], lr: float, steps: int, model=DotSwiGLUModel,
+               ns_iters: int = 5) -> Tuple[List[np.ndarray], List[float]]:
+    """theta_{t+1} = theta_t - lr * NS(grad L(theta_t)) per weight matrix,
+    t = 0..steps-1, full batch.  Returns (theta_steps, losses[t] at theta_t)."""
+    theta = [np.array(w, dtype=np.float64, copy=True) for w in theta0]
+    losses = []
+    for _ in range(steps):
+        losses.append(model.loss(model.forward(K, theta), Vp))
+        g = model.grad(K, Vp, theta)
+        theta = [w - lr * newton_schulz(gw, ns_iters) for w, gw in zip(theta, g)]
     return theta, losses
 
 
