@@ -444,6 +444,20 @@ def run_ours(args, cfg):
         if ttt.check_status(wsw) != 0 or ttt.check_status(wsr) != 0:
             raise SystemExit("device status word set during the write/read split")
         del wsw, wsr
+        # The pages' own inner loop on the whole workload: dot-product loss, Muon
+        # steps (lr 0.1, as the pages give it), same steps and read.
+        ttt.profile_start()
+        ms_mu = time_calls(lambda: ttt.layer_muon(Q, K, V, conv_w, theta0, 0.1, cfg.steps, cfg, theta_out=theta, O=O,
+                                                  workspace=ws))
+        prof_mu = ttt.profile_stop()
+        if ttt.check_status(ws) != 0:
+            raise SystemExit("device status word set during the Muon layer")
+        calls = 5   # time_calls: 2 warm-up + 3 timed
+        paths["dot_loss_muon"] = {
+            "views": cfg.n_views, "lr": 0.1, "steps": cfg.steps, "ms_per_call": round(ms_mu, 3),
+            "tokens_per_s": cfg.n / (ms_mu / 1e3),
+            "ms_per_call_by_kernel": {k: round(r["total_ms"] / calls, 3) for k, r in prof_mu.items()
+                                      if not k.startswith("_") and r["launches"]}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

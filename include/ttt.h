@@ -133,6 +133,38 @@ int ttt_grad(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const 
 int ttt_sgd_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads,
                    float scale, float* theta_out, void* stream);
 
+/* The pages' own inner loop (VGG-T^3, Sec. 3.4, "The dot product loss" and
+ * "TTT MLP Architecture and Inner Optimization"): the dot-product loss
+ * L = -(1/n) sum_i <T_theta(k_i), v'_i> and Muon steps
+ *   theta <- theta - lr * NS5(grad L)   per weight matrix of each head,
+ * NS5 = five cubic Newton-Schulz iterations X <- 1.5 X - 0.5 X X^T X from
+ * X_0 = G / ||G||_F (the pages give 5 iterations and lr 0.1, no polynomial;
+ * the cubic iteration for the orthogonal polar factor is the reading taken,
+ * with no momentum and no shape factor).  The step is scale-free, so the 1/n
+ * of the loss does not matter.  The loss is linear in T's output, so no
+ * forward pass is needed for the gradient.  Fused path only: d in
+ * {16, 32, 64}, h <= 256; wide shapes return TTT_EUNSUPPORTED.  NS5 runs in
+ * FP32; everything else is as in ttt_write.  Workspace: as for ttt_write /
+ * ttt_layer. */
+int ttt_write_muon(const ttt_dims* dims, const uint16_t* K, const uint16_t* V,
+                   const float* conv_w, const float* theta0, float lr, int steps,
+                   float* theta_out, void* workspace, size_t workspace_bytes, void* stream);
+int ttt_layer_muon(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                   const float* conv_w, const float* theta0, float lr, int steps,
+                   float* theta_out, uint16_t* O, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/* The Muon write sharded over processes, as ttt_grad / ttt_sgd_update are for
+ * the mean-squared loss.  ttt_grad_dot: grad = d/dtheta of
+ * -sum_i <T_theta(k_i), vp_i> over the tokens dims describes (workspace of
+ * TTT_OP_WRITE).  ttt_muon_update: theta_out = theta_in - lr * NS5(grads[0] +
+ * ... + grads[n_grads - 1]) per weight matrix of each head, the sum in index
+ * order; theta_out may alias theta_in; no workspace. */
+int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const float* theta,
+                 float* grad, void* workspace, size_t workspace_bytes, void* stream);
+int ttt_muon_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads,
+                    float lr, float* theta_out, void* stream);
+
 /* Read (Eq. 4): O = T_theta(Q) with frozen theta (query mode).  dims describe
  * Q's token count through n_views/grid/n_special; only n, heads, d, h are used. */
 int ttt_read(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O,

@@ -95,7 +95,7 @@ Grids grids_for(const Shape& s, int sms) {
 }
 
 struct Ws {
-  size_t status, w13, w2h, wt, vp, e, part, q, k, v, o, convw, th0, thout, total;
+  size_t status, w13, w2h, wt, vp, e, part, grad, q, k, v, o, convw, th0, thout, total;
   size_t img, acc, z1, z3, da, ab, eb, gemm;   // wide path
 };
 
@@ -144,6 +144,7 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
     w.vp = take(tok_bytes);
     w.e = take(tok_bytes);
     w.part = take(static_cast<size_t>(s.H) * s.slices * g.max_contrib * 3ull * 128 * s.D * 4);
+    w.grad = take(theta_bytes);   // the gradient of a Muon step
   }
   if (op == TTT_OP_LAYER_HOST) {
     w.q = take(tok_bytes);
@@ -560,9 +561,12 @@ struct GradPass {
   long long red_threads;
 };
 
-bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradPass* gp) {
+// dot: the dot-product loss, whose output gradient is the constant -V'; the
+// backward then reads V' where it reads E (no forward pass) and the reduction
+// negates.
+bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradPass* gp, bool dot = false) {
   const Shape& s = c.s;
-  uint16_t* e = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
+  uint16_t* e = dot ? const_cast<uint16_t*>(vp) : reinterpret_cast<uint16_t*>(c.ws + c.w.e);
   unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
   if (!make_token_map(&gp->tk, K, s) || !make_token_map(&gp->tvp, vp, s) || !make_token_map(&gp->tku, K, s, kUnit) ||
       !make_token_map(&gp->teu, e, s, kUnit))
@@ -598,12 +602,13 @@ bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradP
   return true;
 }
 
-// With theta_in: out = theta_in - scale * g (one SGD step).  Without: out = g.
-int run_grad_pass(const Call& c, GradPass& gp, const float* theta, const float* theta_in, float scale, float* out) {
+// With theta_in: out = theta_in - scale * g (one SGD step).  Without: out = scale * g.
+int run_grad_pass(const Call& c, GradPass& gp, const float* theta, const float* theta_in, float scale, float* out,
+                  bool dot = false) {
   const Shape& s = c.s;
   int rc;
   if ((rc = run_pack(s, theta, c.w, c.ws, true, c.st)) != TTT_OK) return rc;
-  if ((rc = launch_fwd<true>(s, gp.tk, gp.tvp, gp.fp, c.g.fwd, c.st)) != TTT_OK) return rc;
+  if (!dot && (rc = launch_fwd<true>(s, gp.tk, gp.tvp, gp.fp, c.g.fwd, c.st)) != TTT_OK) return rc;
   if ((rc = launch_bwd(s, gp.tku, gp.teu, gp.bp, c.g.bwd, c.st)) != TTT_OK) return rc;
   gp.up.theta_in = theta_in;
   gp.up.theta_out = out;
@@ -634,6 +639,53 @@ int run_write(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16
   for (int step = 0; step < steps; ++step) {
     const float* th_in = step == 0 ? theta0 : theta_out;
     if ((rc = run_grad_pass(c, gp, th_in, th_in, scale, theta_out)) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
+// theta_out = theta_in - lr * NS5(sum of n_grads gradients), per (head, matrix).
+int run_muon_update(const Shape& s, const float* theta_in, const float* grads, int n_grads, float lr,
+                    float* theta_out, cudaStream_t st) {
+  MuonParams mp;
+  mp.theta_in = theta_in;
+  mp.grads = grads;
+  mp.theta_out = theta_out;
+  mp.n_grads = n_grads;
+  mp.heads = s.H;
+  mp.d = s.D;
+  mp.h = s.h;
+  mp.lr = lr;
+  const size_t smem = ns_smem_bytes(s.D, s.h);
+  if (cudaFuncSetAttribute(muon_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return TTT_ECUDA;
+  {
+    ProfScope prof(KK_REDUCE, st);
+    muon_update_kernel<<<3 * s.H, kNsThreads, smem, st>>>(mp);
+  }
+  return launch_status();
+}
+
+// The pages' inner loop: `steps` Muon steps on the dot-product loss.
+int run_write_muon(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
+                   const float* theta0, float lr, int steps, float* theta_out) {
+  const Shape& s = c.s;
+  uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
+  float* grad = reinterpret_cast<float*>(c.ws + c.w.grad);
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
+  if (rc != TTT_OK) return rc;
+  if (steps == 0) {
+    if (theta_out != theta0 &&
+        cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return TTT_ECUDA;
+    return TTT_OK;
+  }
+  GradPass gp;
+  if (!setup_grad_pass(c, K, vp, &gp, true)) return TTT_ECUDA;
+  for (int step = 0; step < steps; ++step) {
+    const float* th_in = step == 0 ? theta0 : theta_out;
+    if ((rc = run_grad_pass(c, gp, th_in, nullptr, -1.f, grad, true)) != TTT_OK) return rc;
+    if ((rc = run_muon_update(s, th_in, grad, 1, lr, theta_out, c.st)) != TTT_OK) return rc;
   }
   return TTT_OK;
 }
@@ -794,6 +846,57 @@ int ttt_grad(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const 
   int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
   return run_grad(c, K, Vp, theta, grad);
+}
+
+int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const float* theta, float* grad,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!K || !Vp || !theta || !grad) return TTT_EINVAL;
+  if (!aligned(K) || !aligned(Vp) || !aligned(theta) || !aligned(grad)) return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  if (c.s.wide) return TTT_EUNSUPPORTED;
+  GradPass gp;
+  if (!setup_grad_pass(c, K, Vp, &gp, true)) return TTT_ECUDA;
+  return run_grad_pass(c, gp, theta, nullptr, -1.f, grad, true);
+}
+
+int ttt_muon_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads, float lr,
+                    float* theta_out, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != TTT_OK) return rc;
+  if (s.wide) return TTT_EUNSUPPORTED;
+  if (!theta_in || !grads || !theta_out || n_grads < 1) return TTT_EINVAL;
+  if (!aligned(theta_in) || !aligned(grads) || !aligned(theta_out)) return TTT_EALIGN;
+  return run_muon_update(s, theta_in, grads, n_grads, lr, theta_out, static_cast<cudaStream_t>(stream));
+}
+
+int ttt_write_muon(const ttt_dims* dims, const uint16_t* K, const uint16_t* V, const float* conv_w,
+                   const float* theta0, float lr, int steps, float* theta_out, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!K || !V || !conv_w || !theta0 || !theta_out || steps < 0) return TTT_EINVAL;
+  if (!aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out)) return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  if (c.s.wide) return TTT_EUNSUPPORTED;
+  return run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out);
+}
+
+int ttt_layer_muon(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                   const float* conv_w, const float* theta0, float lr, int steps, float* theta_out, uint16_t* O,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !conv_w || !theta0 || !theta_out || !O || steps < 0) return TTT_EINVAL;
+  if (!aligned(Q) || !aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out) ||
+      !aligned(O))
+    return TTT_EALIGN;
+  Call c;
+  int rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  if (c.s.wide) return TTT_EUNSUPPORTED;
+  if ((rc = run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out)) != TTT_OK) return rc;
+  return run_read(c, Q, theta_out, O);
 }
 
 int ttt_sgd_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads, float scale,

@@ -14,11 +14,16 @@ views, so the views can be split between ranks with no halo:
   rank bit for bit, and the same from run to run;
 * the read of each rank's queries is local.
 
-With one rank this computes what ``ttt_write`` computes.  The exchange is the
-only collective; this module holds only the per-step control flow, and every
-arithmetic step runs in the library's kernels (``cuda_ops``).  ``ShardOps``
-lets the multi-process tests drive the same control flow with other
-operations on CPU ranks.
+With one rank this computes what ``ttt_write`` computes.  The same control
+flow runs the pages' own inner loop (dot-product loss, Muon steps:
+``ttt_grad_dot`` and ``ttt_muon_update``, which orthogonalises the summed
+gradient), ``cuda_ops(dims, inner="muon")``; with one rank that is
+``ttt_write_muon``.
+
+The exchange is the only collective.  This module holds only the per-step
+control flow; every arithmetic step runs in the library's kernels
+(``cuda_ops``).  ``ShardOps`` lets the multi-process tests drive the same
+control flow with other operations on CPU ranks.
 """
 from __future__ import annotations
 
@@ -31,29 +36,43 @@ import torch
 from . import ttt
 
 
+def step_scale(lr: float, n_total: int) -> float:
+    """lr * 2 / n_total in single precision, rounded as the single-process write rounds it."""
+    return float(np.float32(np.float32(lr) * np.float32(2.0)) / np.float32(n_total))
+
+
+def muon_step_size(lr: float, n_total: int) -> float:
+    """Muon's step is scale-free in the gradient: its size is lr itself."""
+    return float(lr)
+
+
 @dataclass
 class ShardOps:
     """The per-rank operations of the sharded layer."""
     conv: Callable[..., torch.Tensor]     # (V, conv_w, dims) -> V'
     grad: Callable[..., torch.Tensor]     # (K, Vp, theta, dims) -> gradient sum of the rank's tokens
-    update: Callable[..., torch.Tensor]   # (theta, grads [world, numel], scale, dims) -> theta'
+    update: Callable[..., torch.Tensor]   # (theta, grads [world, numel], size, dims) -> theta'
     read: Callable[..., torch.Tensor]     # (Q, theta, dims) -> O
+    step_size: Callable[[float, int], float] = step_scale   # (lr, n_total) -> the update's size argument
 
 
-def cuda_ops(dims) -> ShardOps:
-    """The library's kernels, with one write workspace reused by every gradient pass."""
+def cuda_ops(dims, inner: str = "sgd") -> ShardOps:
+    """The library's kernels, with one write workspace reused by every gradient pass.
+    inner = "sgd": mean-squared loss, SGD; "muon": dot-product loss, Muon."""
     ws = ttt.make_workspace(dims, ttt.OP_WRITE)
+    if inner == "sgd":
+        grad, update, size = ttt.grad, ttt.sgd_update, step_scale
+    elif inner == "muon":
+        grad, update, size = ttt.grad_dot, ttt.muon_update, muon_step_size
+    else:
+        raise ValueError(f"unknown inner loop {inner!r}")
     return ShardOps(
         conv=lambda V, conv_w, dm: ttt.shortconv2d(V, conv_w, dm),
-        grad=lambda K, Vp, theta, dm: ttt.grad(K, Vp, theta, dm, workspace=ws),
-        update=lambda theta, grads, scale, dm: ttt.sgd_update(theta, grads, scale, dm),
+        grad=lambda K, Vp, theta, dm: grad(K, Vp, theta, dm, workspace=ws),
+        update=lambda theta, grads, s, dm: update(theta, grads, s, dm),
         read=lambda Q, theta, dm: ttt.read(Q, theta, dm),
+        step_size=size,
     )
-
-
-def step_scale(lr: float, n_total: int) -> float:
-    """lr * 2 / n_total in single precision, rounded as the single-process write rounds it."""
-    return float(np.float32(np.float32(lr) * np.float32(2.0)) / np.float32(n_total))
 
 
 def all_gather_rows(group=None) -> Callable[[torch.Tensor], torch.Tensor]:
@@ -83,7 +102,7 @@ def write_sharded(K, V, conv_w, theta0, lr: float, steps: int, dims, n_total: in
         raise ValueError("steps must be >= 0")
     ops = ops or cuda_ops(dims)
     Vp = ops.conv(V, conv_w, dims)
-    scale = step_scale(lr, n_total)
+    scale = ops.step_size(lr, n_total)
     theta = theta0
     for _ in range(steps):
         g = ops.grad(K, Vp, theta, dims)

@@ -17,13 +17,15 @@ from .inputs import LayerConfig
 __all__ = [
     "TTTError", "Dims", "library_path", "load_library", "workspace_bytes", "make_workspace",
     "shortconv2d", "write", "grad", "sgd_update", "read", "layer", "layer_host", "check_status",
+    "write_muon", "layer_muon", "grad_dot", "muon_update",
     "OP_WRITE", "OP_READ", "OP_LAYER", "OP_LAYER_HOST", "EXPORTED_SYMBOLS", "profile_start", "profile_stop",
 ]
 
 OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
 EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
                     "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
-                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_grad", "ttt_sgd_update")
+                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_grad", "ttt_sgd_update",
+                    "ttt_write_muon", "ttt_layer_muon", "ttt_grad_dot", "ttt_muon_update")
 KERNEL_KINDS = 6
 
 
@@ -82,6 +84,10 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_read.argtypes = [DP, P, P, P, P, S, P]
     lib.ttt_grad.argtypes = [DP, P, P, P, P, P, S, P]
     lib.ttt_sgd_update.argtypes = [DP, P, P, I, F, P, P]
+    lib.ttt_write_muon.argtypes = [DP, P, P, P, P, F, I, P, P, S, P]
+    lib.ttt_layer_muon.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
+    lib.ttt_grad_dot.argtypes = [DP, P, P, P, P, P, S, P]
+    lib.ttt_muon_update.argtypes = [DP, P, P, I, F, P, P]
     lib.ttt_layer.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
     lib.ttt_layer_host.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
     lib.ttt_check_status.argtypes = [P, P]
@@ -94,7 +100,8 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_kernel_name.argtypes = [I]
     lib.ttt_kernel_name.restype = ctypes.c_char_p
     for f in ("ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer", "ttt_layer_host", "ttt_check_status",
-              "ttt_profile_start", "ttt_profile_stop", "ttt_grad", "ttt_sgd_update"):
+              "ttt_profile_start", "ttt_profile_stop", "ttt_grad", "ttt_sgd_update", "ttt_write_muon",
+              "ttt_layer_muon", "ttt_grad_dot", "ttt_muon_update"):
         getattr(lib, f).restype = I
     _LIB = lib
     return lib
@@ -180,6 +187,60 @@ def sgd_update(theta_in, grads, scale: float, dims, theta_out=None) -> torch.Ten
     _check(load_library().ttt_sgd_update(ctypes.byref(dm), _dev(theta_in, torch.float32, "theta_in"),
                                          _dev(grads, torch.float32, "grads"), int(n_grads), float(scale),
                                          _dev(theta_out, torch.float32, "theta_out"), _stream()), "ttt_sgd_update")
+    return theta_out
+
+
+def write_muon(K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, workspace=None) -> torch.Tensor:
+    """theta* after `steps` Muon steps on the dot-product loss (the pages' inner loop)."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta0) if theta_out is None else theta_out
+    ws = make_workspace(dm, OP_WRITE, K.device) if workspace is None else workspace
+    _check(load_library().ttt_write_muon(ctypes.byref(dm), _dev(K, torch.bfloat16, "K"),
+                                         _dev(V, torch.bfloat16, "V"), _dev(conv_w, torch.float32, "conv_w"),
+                                         _dev(theta0, torch.float32, "theta0"), float(lr), int(steps),
+                                         _dev(theta_out, torch.float32, "theta_out"), ws.data_ptr(), ws.numel(),
+                                         _stream()), "ttt_write_muon")
+    return theta_out
+
+
+def layer_muon(Q, K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, O=None,
+               workspace=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The layer with the pages' inner loop (dot-product loss, Muon); returns (theta*, O)."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta0) if theta_out is None else theta_out
+    O = torch.empty_like(Q) if O is None else O
+    ws = make_workspace(dm, OP_LAYER, Q.device) if workspace is None else workspace
+    _check(load_library().ttt_layer_muon(ctypes.byref(dm), _dev(Q, torch.bfloat16, "Q"),
+                                         _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V"),
+                                         _dev(conv_w, torch.float32, "conv_w"), _dev(theta0, torch.float32, "theta0"),
+                                         float(lr), int(steps), _dev(theta_out, torch.float32, "theta_out"),
+                                         _dev(O, torch.bfloat16, "O"), ws.data_ptr(), ws.numel(), _stream()),
+           "ttt_layer_muon")
+    return theta_out, O
+
+
+def grad_dot(K, Vp, theta, dims, out=None, workspace=None) -> torch.Tensor:
+    """d/dtheta of -sum_i <T_theta(k_i), v'_i> over the tokens of (K, Vp)."""
+    dm = Dims.of(dims)
+    out = torch.empty_like(theta) if out is None else out
+    ws = make_workspace(dm, OP_WRITE, K.device) if workspace is None else workspace
+    _check(load_library().ttt_grad_dot(ctypes.byref(dm), _dev(K, torch.bfloat16, "K"),
+                                       _dev(Vp, torch.bfloat16, "Vp"), _dev(theta, torch.float32, "theta"),
+                                       _dev(out, torch.float32, "grad"), ws.data_ptr(), ws.numel(), _stream()),
+           "ttt_grad_dot")
+    return out
+
+
+def muon_update(theta_in, grads, lr: float, dims, theta_out=None) -> torch.Tensor:
+    """theta_out = theta_in - lr * NS5(sum_r grads[r]) per weight matrix; returns theta_out."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta_in) if theta_out is None else theta_out
+    if grads.numel() % theta_in.numel() != 0:
+        raise ValueError("grads must hold whole gradients of theta's size")
+    _check(load_library().ttt_muon_update(ctypes.byref(dm), _dev(theta_in, torch.float32, "theta_in"),
+                                          _dev(grads, torch.float32, "grads"), int(grads.numel() // theta_in.numel()),
+                                          float(lr), _dev(theta_out, torch.float32, "theta_out"), _stream()),
+           "ttt_muon_update")
     return theta_out
 
 

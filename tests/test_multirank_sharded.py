@@ -10,7 +10,9 @@ of the kernels, on a collection of 5 views split 2 + 3.  Checked:
   (the gradient over all tokens is the sum of the shards' sums, Eq. 5);
 * theta* is bit-identical on both ranks (same gathered sums, same order);
 * each rank's read equals the oracle read of its own queries with theta*;
-* steps = 0 returns theta0.
+* steps = 0 returns theta0;
+* the pages' inner loop (dot-product loss, Muon on the summed gradient) run
+  the same way equals the oracle's single-process Muon write.
 """
 import datetime
 import os
@@ -75,6 +77,34 @@ def oracle_ops() -> sharded.ShardOps:
     return sharded.ShardOps(conv=conv, grad=grad, update=update, read=read)
 
 
+def oracle_muon_ops() -> sharded.ShardOps:
+    """The dot-product loss and Muon with the kernels' contracts (ttt_grad_dot returns
+    the gradient of -sum <T(k), v'>, n times the mean loss's; ttt_muon_update takes lr)."""
+    base = oracle_ops()
+
+    def grad(K, Vp, theta, cfg):
+        W1, W3, W2 = _unpack(theta, cfg)
+        g = [np.zeros_like(W1), np.zeros_like(W3), np.zeros_like(W2)]
+        n = K.shape[0]
+        for hd in range(cfg.heads):
+            gh = orc.dot_grad(K[:, hd].numpy(), Vp[:, hd].numpy(), W1[hd], W3[hd], W2[hd])
+            for m in range(3):
+                g[m][hd] = gh[m] * n
+        return _pack(*g)
+
+    def update(theta, grads, lr, cfg):
+        total = grads[0].clone()
+        for r in range(1, grads.shape[0]):
+            total += grads[r]
+        G = _unpack(total, cfg)
+        W = _unpack(theta, cfg)
+        new = [np.stack([W[m][hd] - lr * orc.newton_schulz(G[m][hd]) for hd in range(cfg.heads)]) for m in range(3)]
+        return _pack(*new)
+
+    return sharded.ShardOps(conv=base.conv, grad=grad, update=update, read=base.read,
+                            step_size=sharded.muon_step_size)
+
+
 def _gloo_gather(t):
     parts = [torch.empty_like(t.reshape(-1)) for _ in range(dist.get_world_size())]
     dist.all_gather(parts, t.reshape(-1).contiguous())
@@ -101,7 +131,10 @@ def _worker(rank: int, world: int, port: int, q) -> None:
                                          _gloo_gather, ops)
         theta_ranks = _gloo_gather(theta)
         th_zero = sharded.write_sharded(K, V, inp["conv_w"], th0, CFG.lr, 0, local, CFG.n, _gloo_gather, ops)
-        q.put((rank, theta.numpy(), O.numpy(), theta_ranks.numpy(), bool(torch.equal(th_zero, th0))))
+        th_muon = sharded.write_sharded(K, V, inp["conv_w"], th0, 0.1, 2, local, CFG.n, _gloo_gather,
+                                        oracle_muon_ops())
+        q.put((rank, theta.numpy(), O.numpy(), theta_ranks.numpy(), bool(torch.equal(th_zero, th0)),
+               th_muon.numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -132,7 +165,7 @@ def test_sharded_write_two_gloo_ranks_matches_single_process_oracle():
     ref_flat = _pack(*ref).numpy()
     th0_flat = _pack(*th0).numpy()
 
-    (_, th_a, O_a, ranks_a, zero_a), (_, th_b, O_b, ranks_b, zero_b) = results
+    (_, th_a, O_a, ranks_a, zero_a, mu_a), (_, th_b, O_b, ranks_b, zero_b, mu_b) = results
     assert np.array_equal(th_a, th_b) and np.array_equal(ranks_a[0], ranks_a[1])
     assert zero_a and zero_b
     delta, delta_ref = th_a - th0_flat, ref_flat - th0_flat
@@ -145,3 +178,13 @@ def test_sharded_write_two_gloo_ranks_matches_single_process_oracle():
         Qr = Qall[a * tpv:b * tpv]
         O_ref = np.stack([orc.read(Qr[:, hd], W[0][hd], W[1][hd], W[2][hd]) for hd in range(H)], axis=1)
         assert np.max(np.abs(O - O_ref)) <= 1e-12 * np.max(np.abs(O_ref))
+
+    # the pages' inner loop, sharded the same way: the oracle's Muon write over all views
+    assert np.array_equal(mu_a, mu_b)
+    mref = [np.zeros_like(w) for w in th0]
+    for hd in range(H):
+        th, _ = orc.muon_write(K[:, hd], Vp[:, hd], [w[hd] for w in th0], 0.1, 2)
+        for m in range(3):
+            mref[m][hd] = th[m]
+    mref_flat = _pack(*mref).numpy()
+    assert np.max(np.abs(mu_a - mref_flat)) <= 1e-10 * np.max(np.abs(mref_flat - th0_flat))
