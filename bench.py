@@ -458,6 +458,22 @@ def run_ours(args, cfg):
             "tokens_per_s": cfg.n / (ms_mu / 1e3),
             "ms_per_call_by_kernel": {k: round(r["total_ms"] / calls, 3) for k, r in prof_mu.items()
                                       if not k.startswith("_") and r["launches"]}}
+        # The same layer with Q, K, V left in pinned host memory and streamed in
+        # chunks of 100 views (the offload path for collections beyond HBM).
+        from test_layer_reconstruction_b200 import stream as tstream
+        hq, hk, hv = (t.cpu().pin_memory() for t in (Q, K, V))
+        chunk = min(100, cfg.n_views)
+
+        def streamed_call():
+            th_ = tstream.write_streamed(hk, hv, conv_w, theta0, cfg.lr, cfg.steps, cfg, chunk)
+            tstream.read_streamed(hq, th_, cfg, chunk)
+
+        ms_st = time_calls(streamed_call, reps=2, warm=1)
+        paths["streamed_from_host"] = {
+            "views": cfg.n_views, "chunk_views": chunk, "ms_per_call": round(ms_st, 1),
+            "tokens_per_s": cfg.n / (ms_st / 1e3),
+            "host_bytes_per_call": int((cfg.steps * 2 + 2) * hq.numel() * 2)}
+        del hq, hk, hv
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

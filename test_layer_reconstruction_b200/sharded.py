@@ -50,7 +50,7 @@ def muon_step_size(lr: float, n_total: int) -> float:
 class ShardOps:
     """The per-rank operations of the sharded layer."""
     conv: Callable[..., torch.Tensor]     # (V, conv_w, dims) -> V'
-    grad: Callable[..., torch.Tensor]     # (K, Vp, theta, dims) -> gradient sum of the rank's tokens
+    grad: Callable[..., torch.Tensor]     # (K, Vp, theta, dims, out=None) -> gradient sum of the tokens
     update: Callable[..., torch.Tensor]   # (theta, grads [world, numel], size, dims) -> theta'
     read: Callable[..., torch.Tensor]     # (Q, theta, dims) -> O
     step_size: Callable[[float, int], float] = step_scale   # (lr, n_total) -> the update's size argument
@@ -68,7 +68,7 @@ def cuda_ops(dims, inner: str = "sgd") -> ShardOps:
         raise ValueError(f"unknown inner loop {inner!r}")
     return ShardOps(
         conv=lambda V, conv_w, dm: ttt.shortconv2d(V, conv_w, dm),
-        grad=lambda K, Vp, theta, dm: grad(K, Vp, theta, dm, workspace=ws),
+        grad=lambda K, Vp, theta, dm, out=None: grad(K, Vp, theta, dm, out=out, workspace=ws),
         update=lambda theta, grads, s, dm: update(theta, grads, s, dm),
         read=lambda Q, theta, dm: ttt.read(Q, theta, dm),
         step_size=size,

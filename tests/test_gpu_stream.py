@@ -1,0 +1,66 @@
+"""GPU parity of the host-streamed layer (K, V, Q in pinned host memory,
+chunks of whole views brought to the device one at a time).
+
+* One chunk: the streamed write equals ttt_write, and with the pages' inner
+  loop ttt_write_muon, bit for bit (same kernels, same reduction order).
+* Chunks of 5 views over 24 (the last one 4): one step at lr 50 matches the
+  single-pass write up to summation order (5e-4 of the step); at the
+  workload's step size theta* is within two units in the last place plus the
+  step's summation-order difference; the Muon write within 1e-4 of its step.
+* The streamed read equals ttt_read bit for bit, with a ragged last chunk.
+"""
+import pytest
+import torch
+
+from test_layer_reconstruction_b200 import inputs as tin
+from test_layer_reconstruction_b200 import stream, ttt
+from ttt_testlib import normwise
+
+pytestmark = pytest.mark.gpu
+
+CFG = tin.CONFIGS["views24_37x37p5_h16_d64_h256"]
+
+
+def _inputs(cfg):
+    inp = tin.make_inputs(cfg)
+    host = {k: inp[k].to(torch.bfloat16).contiguous().pin_memory() for k in ("Q", "K", "V")}
+    dev = {k: host[k].cuda() for k in host}
+    dev["conv_w"] = inp["conv_w"].float().contiguous().cuda()
+    dev["theta"] = tin.pack_theta(inp["W1"], inp["W3"], inp["W2"]).cuda()
+    return host, dev
+
+
+def test_one_chunk_equals_single_pass_bitwise():
+    host, dev = _inputs(CFG)
+    for inner, write in (("sgd", ttt.write), ("muon", ttt.write_muon)):
+        lr = CFG.lr if inner == "sgd" else 0.1
+        full = write(dev["K"], dev["V"], dev["conv_w"], dev["theta"], lr, 2, CFG)
+        st = stream.write_streamed(host["K"], host["V"], dev["conv_w"], dev["theta"], lr, 2, CFG, CFG.n_views, inner)
+        torch.cuda.synchronize()
+        assert torch.equal(full, st), inner
+
+
+def test_chunked_write_matches_single_pass():
+    host, dev = _inputs(CFG)
+    th0 = dev["theta"].double().cpu().numpy()
+    big = stream.write_streamed(host["K"], host["V"], dev["conv_w"], dev["theta"], 50.0, 1, CFG, 5)
+    full_big = ttt.write(dev["K"], dev["V"], dev["conv_w"], dev["theta"], 50.0, 1, CFG)
+    torch.cuda.synchronize()
+    assert normwise(big.double().cpu().numpy() - th0, full_big.double().cpu().numpy() - th0) <= 5e-4
+    theta = stream.write_streamed(host["K"], host["V"], dev["conv_w"], dev["theta"], CFG.lr, 2, CFG, 5)
+    full = ttt.write(dev["K"], dev["V"], dev["conv_w"], dev["theta"], CFG.lr, 2, CFG)
+    torch.cuda.synchronize()
+    step = (full - dev["theta"]).abs().max()
+    assert bool(((theta - full).abs() <= full.abs() * 2.0 ** -22 + 1e-4 * step).all())
+    mu = stream.write_streamed(host["K"], host["V"], dev["conv_w"], dev["theta"], 0.1, 2, CFG, 5, "muon")
+    mu_full = ttt.write_muon(dev["K"], dev["V"], dev["conv_w"], dev["theta"], 0.1, 2, CFG)
+    torch.cuda.synchronize()
+    assert normwise(mu.double().cpu().numpy() - th0, mu_full.double().cpu().numpy() - th0) <= 1e-4
+
+
+def test_streamed_read_equals_read():
+    host, dev = _inputs(CFG)
+    O = stream.read_streamed(host["Q"], dev["theta"], CFG, 7)
+    ref = ttt.read(dev["Q"], dev["theta"], CFG)
+    torch.cuda.synchronize()
+    assert O.is_pinned() and torch.equal(O, ref.cpu())
