@@ -6,7 +6,8 @@ chunks of whole views brought to the device one at a time).
 * Chunks of 5 views over 24 (the last one 4): one step at lr 50 matches the
   single-pass write up to summation order (5e-4 of the step); at the
   workload's step size theta* is within two units in the last place plus the
-  step's summation-order difference; the Muon write within 1e-4 of its step.
+  step's summation-order difference; the Muon write within 8 x 5e-4 of its
+  step (NS5 magnifies a gradient difference at most 1.5^5 times).
 * The streamed read equals ttt_read bit for bit, with a ragged last chunk.
 """
 import pytest
@@ -52,10 +53,15 @@ def test_chunked_write_matches_single_pass():
     torch.cuda.synchronize()
     step = (full - dev["theta"]).abs().max()
     assert bool(((theta - full).abs() <= full.abs() * 2.0 ** -22 + 1e-4 * step).all())
+    # Muon: the chunked gradient sum differs from the single pass by summation
+    # order (within the 5e-4 checked above); NS5's derivative on the normalised
+    # singular values is at most 1.5^5 < 8, so the two steps agree within
+    # 8 x 5e-4.  (After the first step the two thetas may differ in the last
+    # place, which can round a bf16 operand of the second step differently.)
     mu = stream.write_streamed(host["K"], host["V"], dev["conv_w"], dev["theta"], 0.1, 2, CFG, 5, "muon")
     mu_full = ttt.write_muon(dev["K"], dev["V"], dev["conv_w"], dev["theta"], 0.1, 2, CFG)
     torch.cuda.synchronize()
-    assert normwise(mu.double().cpu().numpy() - th0, mu_full.double().cpu().numpy() - th0) <= 1e-4
+    assert normwise(mu.double().cpu().numpy() - th0, mu_full.double().cpu().numpy() - th0) <= 8 * 5e-4
 
 
 def test_streamed_read_equals_read():
