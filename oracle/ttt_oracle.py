@@ -46,6 +46,18 @@ build, pinned here before any kernel) takes these readings:
   X <- 1.5 X - 0.5 X X^T X, five times; then theta <- theta - lr * X_5.  No
   momentum (one or two steps), no shape factor.
 
+The layer's surround (QKV projections, Q/K normalisation, output projection;
+a later step of the build, pinned here first) takes these readings:
+
+* Projections (Eq. 1 of [summary] Sec. 3, "QKV projection with
+  normalization"), in row-vector form: q = x Wq, k = x Wk, v = x Wv with
+  [C, C] matrices, C = heads * d, split into heads of d channels; the output
+  projection ("the output projection matrices that follow the attention
+  operation") is out = o Wo.  No biases (none are given).
+* LN_q and LN_k are replaced by L2 normalisation ("The LayerNorm removal":
+  k_hat = k / ||k||_2) of each (token, head) row of length d; V is not
+  normalised.  A zero row stays zero.
+
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against
 facts that do not come from this file (library routines, finite differences,
 closed forms, brute force, invariants).
@@ -61,6 +73,7 @@ __all__ = [
     "Dims", "shortconv2d", "sigmoid", "swiglu_forward", "mse_loss", "mse_grad", "mse_grad_chunked",
     "sgd_write", "read", "layer", "LinearModel", "SwiGLUModel", "ChunkedSwiGLUModel",
     "dot_loss", "dot_grad", "newton_schulz", "muon_write", "DotSwiGLUModel", "DotLinearModel",
+    "l2_normalize_heads", "ttt_attention",
 ]
 
 
@@ -326,6 +339,53 @@ def muon_write(K, Vp, theta0: Sequence[np.ndarray], lr: float, steps: int, model
 def read(Q, W1, W3, W2) -> np.ndarray:
     """o_i = T_theta(q_i) for every row of Q [n, d]."""
     return swiglu_forward(Q, W1, W3, W2)[0]
+
+
+# ---------------------------------------------------------------------------
+# The layer's surround ([summary] Sec. 3 "QKV projection with normalization",
+# Eq. 1; Sec. 3.2 / "The LayerNorm removal"; the output projection)
+# ---------------------------------------------------------------------------
+
+def l2_normalize_heads(Y: np.ndarray, heads: int) -> np.ndarray:
+    """Y [n, heads*d] with every (token, head) row of length d scaled to unit
+    L2 norm; rows of norm zero stay zero.  Returns [n, heads, d]."""
+    Y = np.asarray(Y, np.float64)
+    n = Y.shape[0]
+    R = Y.reshape(n, heads, -1)
+    nrm = np.sqrt(np.sum(R * R, axis=2, keepdims=True))
+    return np.divide(R, nrm, out=np.zeros_like(R), where=nrm > 0)
+
+
+def ttt_attention(X, Wq, Wk, Wv, Wo, conv_w, W1, W3, W2, lr: float, steps: int, dims: Dims, inner: str = "sgd"):
+    """The global attention layer with the TTT layer in place of softmax
+    attention: q_hat = L2(X Wq), k_hat = L2(X Wk) per head, v = X Wv; the
+    layer on (q_hat, k_hat, v) with ``inner`` = "sgd" (mean-squared loss, SGD)
+    or "muon" (dot-product loss, Muon); out = O Wo.
+
+    X: [n, C]; Wq, Wk, Wv, Wo: [C, C]; the rest as for ``layer``.
+    Returns (out [n, C], W1*, W3*, W2*)."""
+    X = np.asarray(X, np.float64)
+    H = np.asarray(W1).shape[0]
+    n = X.shape[0]
+    Q = l2_normalize_heads(X @ Wq, H)
+    K = l2_normalize_heads(X @ Wk, H)
+    V = (X @ Wv).reshape(n, H, -1)
+    if inner == "sgd":
+        W1s, W3s, W2s, O, _ = layer(Q, K, V, conv_w, W1, W3, W2, lr, steps, dims)
+    elif inner == "muon":
+        d = V.shape[2]
+        Vp = shortconv2d(V.reshape(n, H * d), conv_w, dims).reshape(n, H, d)
+        W1s, W3s, W2s = [], [], []
+        O = np.zeros_like(Q)
+        for hd in range(H):
+            th, _ = muon_write(K[:, hd], Vp[:, hd], (np.asarray(W1[hd], np.float64), np.asarray(W3[hd], np.float64),
+                                                     np.asarray(W2[hd], np.float64)), lr, steps)
+            W1s.append(th[0]); W3s.append(th[1]); W2s.append(th[2])
+            O[:, hd] = read(Q[:, hd], *th)
+        W1s, W3s, W2s = np.stack(W1s), np.stack(W3s), np.stack(W2s)
+    else:
+        raise ValueError(f"unknown inner loop {inner!r}")
+    return O.reshape(n, -1) @ Wo, W1s, W3s, W2s
 
 
 def layer(Q, K, V, conv_w, W1, W3, W2, lr: float, steps: int, dims: Dims):
