@@ -776,6 +776,14 @@ uint8_t* noalloc_scratch() {
   return static_cast<uint8_t*>(addr[dev]);
 }
 
+// Host-only shape check of the entry points that have no wide-head path.
+int fused_only(const ttt_dims* dims) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != TTT_OK) return rc;
+  return s.wide ? TTT_EUNSUPPORTED : TTT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -852,10 +860,11 @@ int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, co
                  void* workspace, size_t workspace_bytes, void* stream) {
   if (!K || !Vp || !theta || !grad) return TTT_EINVAL;
   if (!aligned(K) || !aligned(Vp) || !aligned(theta) || !aligned(grad)) return TTT_EALIGN;
-  Call c;
-  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  int rc = fused_only(dims);
   if (rc != TTT_OK) return rc;
-  if (c.s.wide) return TTT_EUNSUPPORTED;
+  Call c;
+  rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
   GradPass gp;
   if (!setup_grad_pass(c, K, Vp, &gp, true)) return TTT_ECUDA;
   return run_grad_pass(c, gp, theta, nullptr, -1.f, grad, true);
@@ -863,10 +872,10 @@ int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, co
 
 int ttt_muon_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads, float lr,
                     float* theta_out, void* stream) {
-  Shape s;
-  int rc = check_dims(dims, &s);
+  int rc = fused_only(dims);
   if (rc != TTT_OK) return rc;
-  if (s.wide) return TTT_EUNSUPPORTED;
+  Shape s;
+  check_dims(dims, &s);
   if (!theta_in || !grads || !theta_out || n_grads < 1) return TTT_EINVAL;
   if (!aligned(theta_in) || !aligned(grads) || !aligned(theta_out)) return TTT_EALIGN;
   return run_muon_update(s, theta_in, grads, n_grads, lr, theta_out, static_cast<cudaStream_t>(stream));
@@ -877,10 +886,11 @@ int ttt_write_muon(const ttt_dims* dims, const uint16_t* K, const uint16_t* V, c
                    size_t workspace_bytes, void* stream) {
   if (!K || !V || !conv_w || !theta0 || !theta_out || steps < 0) return TTT_EINVAL;
   if (!aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out)) return TTT_EALIGN;
-  Call c;
-  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  int rc = fused_only(dims);
   if (rc != TTT_OK) return rc;
-  if (c.s.wide) return TTT_EUNSUPPORTED;
+  Call c;
+  rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
   return run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out);
 }
 
@@ -891,10 +901,11 @@ int ttt_layer_muon(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, c
   if (!aligned(Q) || !aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out) ||
       !aligned(O))
     return TTT_EALIGN;
-  Call c;
-  int rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
+  int rc = fused_only(dims);
   if (rc != TTT_OK) return rc;
-  if (c.s.wide) return TTT_EUNSUPPORTED;
+  Call c;
+  rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
   if ((rc = run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out)) != TTT_OK) return rc;
   return run_read(c, Q, theta_out, O);
 }

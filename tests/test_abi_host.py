@@ -69,3 +69,30 @@ def test_host_validation_codes(lib):
 def test_workspace_bytes_rejects_bad_dims(lib):
     assert lib.ttt_workspace_bytes(ctypes.byref(_dims(d=48)), 0) == 0
     assert lib.ttt_workspace_bytes(ctypes.byref(_dims()), 7) == 0
+
+
+def test_host_validation_codes_of_the_sharded_muon_and_host_entry_points(lib):
+    dm = ctypes.byref(_dims())
+    wide = ctypes.byref(_dims(d=128, h=192))
+    # gradient passes of the sharded write
+    for fn in (lib.ttt_grad, lib.ttt_grad_dot):
+        assert fn(dm, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+        assert fn(dm, FAKE, FAKE, FAKE_MIS, FAKE, FAKE, 1 << 20, None) == -2
+        assert fn(ctypes.byref(_dims(d=48)), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == -3
+    assert lib.ttt_grad_dot(wide, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == -3   # no wide Muon path
+    # updates
+    assert lib.ttt_sgd_update(dm, FAKE, FAKE, 0, 1.0, FAKE, None) == -1               # no gradients
+    assert lib.ttt_sgd_update(dm, None, FAKE, 1, 1.0, FAKE, None) == -1
+    assert lib.ttt_sgd_update(dm, FAKE, FAKE_MIS, 1, 1.0, FAKE, None) == -2
+    assert lib.ttt_muon_update(dm, FAKE, FAKE, 0, 0.1, FAKE, None) == -1
+    assert lib.ttt_muon_update(wide, FAKE, FAKE, 1, 0.1, FAKE, None) == -3
+    # the Muon write and layer
+    assert lib.ttt_write_muon(dm, FAKE, FAKE, FAKE, FAKE, 0.1, -1, FAKE, FAKE, 1 << 20, None) == -1
+    assert lib.ttt_write_muon(dm, FAKE_MIS, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, 1 << 20, None) == -2
+    assert lib.ttt_write_muon(wide, FAKE, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, 1 << 20, None) == -3
+    assert lib.ttt_layer_muon(dm, None, FAKE, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert lib.ttt_layer_muon(wide, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None) == -3
+    # host buffers
+    assert lib.ttt_layer_host(dm, None, FAKE, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert lib.ttt_layer_host(dm, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, -1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+
