@@ -96,7 +96,10 @@ def write_sharded(K, V, conv_w, theta0, lr: float, steps: int, dims, n_total: in
     K, V hold this rank's views (``dims`` describes them); ``n_total`` is the
     collection's token count over all ranks; ``gather`` returns every rank's
     tensor stacked in rank order.  Every rank must call this with the same
-    ``theta0``, ``lr``, ``steps`` and ``n_total``.
+    ``theta0``, ``lr``, ``steps`` and ``n_total``.  If the exchange fails (a
+    rank has left, or the process group's timeout ran out), the call raises
+    RuntimeError naming the step; no collective is left half-issued on the
+    ranks that remain, since each step issues exactly one.
     """
     if steps < 0:
         raise ValueError("steps must be >= 0")
@@ -104,9 +107,13 @@ def write_sharded(K, V, conv_w, theta0, lr: float, steps: int, dims, n_total: in
     Vp = ops.conv(V, conv_w, dims)
     scale = ops.step_size(lr, n_total)
     theta = theta0
-    for _ in range(steps):
+    for step in range(steps):
         g = ops.grad(K, Vp, theta, dims)
-        theta = ops.update(theta, gather(g), scale, dims)
+        try:
+            gathered = gather(g)
+        except Exception as exc:   # a rank that left, or the process group's timeout
+            raise RuntimeError(f"sharded write: the gradient exchange of step {step} failed: {exc}") from exc
+        theta = ops.update(theta, gathered, scale, dims)
     return theta.clone() if steps == 0 else theta
 
 

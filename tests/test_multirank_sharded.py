@@ -188,3 +188,46 @@ def test_sharded_write_two_gloo_ranks_matches_single_process_oracle():
             mref[m][hd] = th[m]
     mref_flat = _pack(*mref).numpy()
     assert np.max(np.abs(mu_a - mref_flat)) <= 1e-10 * np.max(np.abs(mref_flat - th0_flat))
+
+
+def _failing_worker(rank: int, world: int, port: int, q) -> None:
+    """Rank 1 leaves after its gradient, before the first exchange; rank 0 must
+    get an error from the exchange, not hang."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=20))
+    a, b = SPLIT[rank]
+    local = CFG.with_views(b - a)
+    inp = tin.make_inputs(CFG, views=range(a, b))
+    K, V = (inp[k].double() for k in ("K", "V"))
+    th0 = tin.pack_theta(inp["W1"], inp["W3"], inp["W2"]).double()
+    if rank == 1:
+        q.put((rank, "left"))
+        q.close()
+        q.join_thread()   # the message is out before the process vanishes
+        os._exit(0)       # gone without a word: no destroy, no collective
+    try:
+        sharded.write_sharded(K, V, inp["conv_w"], th0, CFG.lr, 2, local, CFG.n, _gloo_gather, oracle_ops())
+        q.put((rank, "no error"))
+    except RuntimeError as exc:
+        q.put((rank, str(exc)))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_sharded_write_reports_a_rank_that_left():
+    import time
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    t0 = time.monotonic()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert results[1] == "left"
+    assert "gradient exchange of step 0 failed" in results[0], results[0]
+    assert time.monotonic() - t0 < 120
+
