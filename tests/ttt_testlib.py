@@ -94,3 +94,26 @@ def compare_O(O_gpu: torch.Tensor, ref, heads=None, rows=None):
             r, g = r[rows], g[rows]
         worst = max(worst, normwise(g, r))
     return worst
+
+
+# ---------------------------------------------------------------- guard bands
+GUARD = 4096          # bytes of canary on each side (keeps the payload 256-byte aligned)
+CANARY = 0xA5
+
+
+def guarded(shape, dtype, device, fill=None):
+    """A tensor of `shape` inside a byte buffer with GUARD canary bytes on both
+    sides.  Returns (payload view, whole buffer).  `fill` poisons the payload
+    (e.g. NaN for outputs)."""
+    nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((GUARD + nbytes + GUARD,), CANARY, dtype=torch.uint8, device=device)
+    view = buf[GUARD:GUARD + nbytes].view(dtype).reshape(shape)
+    if fill is not None:
+        view.fill_(fill)
+    return view, buf
+
+
+def guards_intact(buf) -> bool:
+    """True when both canary bands of a `guarded` buffer are untouched."""
+    b = buf.cpu()
+    return bool((b[:GUARD] == CANARY).all()) and bool((b[-GUARD:] == CANARY).all())
