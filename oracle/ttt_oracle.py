@@ -32,8 +32,7 @@ Readings taken where the pages are silent or disagree:
   bias, depthwise over all heads*d channels, weights shared by all views.
 * Special tokens are the first ``n_special`` tokens of each view.
 
-The pages' own inner loop (dot-product loss and Muon; a later step of the
-build, pinned here before any kernel) takes these readings:
+The pages' own inner loop (dot-product loss and Muon) takes these readings:
 
 * Dot-product loss ([summary] Sec. 3.4, "The dot product loss": the per-token
   loss is T(k)^T v, and the arg-min form implies a minus sign):
@@ -46,8 +45,8 @@ build, pinned here before any kernel) takes these readings:
   X <- 1.5 X - 0.5 X X^T X, five times; then theta <- theta - lr * X_5.  No
   momentum (one or two steps), no shape factor.
 
-The layer's surround (QKV projections, Q/K normalisation, output projection;
-a later step of the build, pinned here first) takes these readings:
+The layer's surround (QKV projections, Q/K normalisation, output projection)
+takes these readings:
 
 * Projections (Eq. 1 of [summary] Sec. 3, "QKV projection with
   normalization"), in row-vector form: q = x Wq, k = x Wk, v = x Wv with
