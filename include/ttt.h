@@ -229,7 +229,10 @@ const char* ttt_status_str(int status);
  * ttt_profile_stop synchronises those events and fills, per kernel kind k
  * (0 <= k < TTT_KERNEL_KINDS, named by ttt_kernel_name), the number of
  * launches and their summed device time in milliseconds.  At most 65536
- * launches are recorded per session; later ones are counted in `dropped`. */
+ * launches are recorded per session; later ones are counted in `dropped`.
+ * The "reduce_sgd" kind covers every theta-sized step kernel: the split-K
+ * reduction with its SGD step, the fixed-order update of ttt_sgd_update and
+ * the Newton-Schulz step of the Muon entry points. */
 #define TTT_KERNEL_KINDS 6
 typedef struct ttt_kernel_times {
   int32_t launches[TTT_KERNEL_KINDS];
