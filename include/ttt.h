@@ -215,6 +215,18 @@ int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t*
 int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O,
                      void* stream);
 
+/* The device status of ttt_read_noalloc, which has no workspace to pass to
+ * ttt_check_status: synchronises `stream`, then reads the status word that
+ * the read's kernels keep at the start of the fixed scratch array of the
+ * current device.  Returns TTT_OK, TTT_EDEVICE if a kernel recorded a fault
+ * (a bounded wait that ran out; the word is then cleared and the read's O
+ * must not be used), or TTT_ECUDA.  Each ttt_read_noalloc clears the word
+ * when it starts, so call this after the read and before the next one on the
+ * device.  Allocates nothing.  The array's device address is looked up once
+ * per device; after cudaDeviceReset neither this call nor ttt_read_noalloc
+ * may be used again in the process. */
+int ttt_read_noalloc_status(void* stream);
+
 /* Synchronises `stream`, then reads the device status word of `workspace`:
  * TTT_OK, TTT_EDEVICE if a kernel recorded a fault (the word is cleared), or
  * TTT_ECUDA. */

@@ -801,6 +801,20 @@ int ttt_trace_read(unsigned long long* out, int reset) {
 }
 #endif
 
+int ttt_read_noalloc_status(void* stream) {
+  uint8_t* scratch = noalloc_scratch();
+  if (!scratch) return TTT_ECUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TTT_ECUDA;
+  // The status word is the first field of every workspace layout (offset 0).
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ECUDA;
+  if (v != 0) {
+    if (cudaMemset(scratch, 0, sizeof(v)) != cudaSuccess) return TTT_ECUDA;
+    return TTT_EDEVICE;
+  }
+  return TTT_OK;
+}
+
 int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta, uint16_t* O, void* stream) {
   if (!Q || !theta || !O) return TTT_EINVAL;
   if (!aligned(Q) || !aligned(theta) || !aligned(O)) return TTT_EALIGN;

@@ -12,21 +12,25 @@ then the ``grid_h x grid_w`` patch grid in row-major order):
 * VGG-T^3 paper, Sec. 3.2 / App. A: per-head width 64 (VGGT width 1024 = 16 x 64),
   SwiGLU fast-weight MLP, 1 inner step for short collections and 2 at 1k views.
 
-Distributions.  In the layer, Q, K and V are projections of the same token
-features, so V at a token is partly predictable from K at that token.  The
-draws keep that structure: every (token, head) row has one latent x ~ N(0, I_d),
-and with per-head projections P_Q, P_K, P_V ~ N(0, 1/d) (d x d, one draw per
-sequence)
-    K = x P_K / ||x P_K||,  Q = x P_Q / ||x P_Q||   (the pages' L2 normalisation
-                                                     of Q and K, Sec. 3.2)
-    V = x P_V                                       (rows of unit variance),
-each then rounded to bfloat16.  Depthwise 3x3 weights ~ N(0, 1/9); fast
-weights Xavier-normal with std sqrt(2 / (d + h)).
+Distributions.  The workloads' own draws ("stated", the default): every
+(token, head) row of K and of Q is an N(0, I_d) draw divided by its Euclidean
+norm (the pages' L2 normalisation of queries and keys, Sec. 3.4 "The
+LayerNorm removal"), V ~ N(0, 1) elementwise, all three independent, each then
+rounded to bfloat16 (round-to-nearest-even).  Depthwise 3x3 weights ~
+N(0, 1/9); fast weights Xavier-normal with std sqrt(2 / (d + h)).
 
-Every view's latents are drawn from their own generator, seeded by a
-SplitMix64 mix of (seed, tensor id, view index), so any subset or permutation
-of views reproduces the same values.  Held-out views draw their latents from
-the held-out seed and share the sequence's projections.
+A second family ("correlated") gives the tokens the structure of projections
+of one token feature, as in the attention layer the TTT layer replaces: every
+(token, head) row has one latent x ~ N(0, I_d), and with per-head projections
+P_Q, P_K, P_V ~ N(0, 1/d) (d x d, one draw per sequence)
+    K = x P_K / ||x P_K||,  Q = x P_Q / ||x P_Q||,  V = x P_V,
+so V at a token is linearly predictable from K at that token.  It is an extra
+parity case, selected per workload with ``LayerConfig.draws``.
+
+Every view's rows are drawn from their own generator, seeded by a SplitMix64
+mix of (seed, tensor id, view index), so any subset or permutation of views
+reproduces the same values.  Held-out views use the held-out seed (with the
+correlated family they draw new latents and share the sequence's projections).
 """
 from __future__ import annotations
 
@@ -89,6 +93,7 @@ class LayerConfig:
     fp32_inputs: bool = False      # the tiny case draws fp32 Q/K/V
     heldout_views: int = 0         # frozen-theta read of extra views
     heldout_seed: int = 0
+    draws: str = "stated"          # "stated" (independent) or "correlated"
 
     @property
     def tokens_per_view(self) -> int:
@@ -100,6 +105,9 @@ class LayerConfig:
 
     def with_views(self, n_views: int) -> "LayerConfig":
         return dataclasses.replace(self, n_views=n_views)
+
+    def with_draws(self, draws: str) -> "LayerConfig":
+        return dataclasses.replace(self, draws=draws)
 
     def flops(self) -> float:
         """Algorithmic FLOPs of conv-free layer math: (14*steps + 6) * d * h per token and head."""
@@ -159,6 +167,20 @@ def _project(X, P, normalise) -> torch.Tensor:
     return out
 
 
+def _unit_rows(cfg, views, device, seed, tensor_id) -> torch.Tensor:
+    """N(0, I_d) rows divided by their norm, drawn view by view."""
+    parts = []
+    for v in views:
+        r = _randn((cfg.tokens_per_view, cfg.heads, cfg.d), seed, tensor_id, v, device)
+        parts.append(r / torch.linalg.vector_norm(r, dim=-1, keepdim=True))
+    return torch.cat(parts, 0) if parts else torch.zeros(0, cfg.heads, cfg.d, device=device)
+
+
+def _normal_rows(cfg, views, device, seed, tensor_id) -> torch.Tensor:
+    parts = [_randn((cfg.tokens_per_view, cfg.heads, cfg.d), seed, tensor_id, v, device) for v in views]
+    return torch.cat(parts, 0) if parts else torch.zeros(0, cfg.heads, cfg.d, device=device)
+
+
 def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] = None,
                 heldout: bool = False) -> Dict[str, torch.Tensor]:
     """Draw the layer's inputs.
@@ -168,19 +190,28 @@ def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] =
     W1, W3 [heads, d, h]; W2 [heads, h, d].  ``views`` selects (and orders) the
     views drawn; ``heldout`` draws the held-out query views instead (Q only).
     """
+    if cfg.draws not in ("stated", "correlated"):
+        raise ValueError(f"unknown draws {cfg.draws!r}")
     if views is None:
         views = range(cfg.heldout_views if heldout else cfg.n_views)
     views = list(views)
     seed = cfg.heldout_seed if heldout else cfg.seed
     out: Dict[str, torch.Tensor] = {}
     rnd = (lambda t: t) if cfg.fp32_inputs else bf16_round
-    X = _latents(cfg, views, device, seed)
-    out["Q"] = rnd(_project(X, _projection(cfg, _TID_Q, device), True))
-    if heldout:
-        return out
-    out["K"] = rnd(_project(X, _projection(cfg, _TID_K, device), True))
-    out["V"] = rnd(_project(X, _projection(cfg, _TID_V, device), False))
-    del X
+    if cfg.draws == "stated":
+        out["Q"] = rnd(_unit_rows(cfg, views, device, seed, _TID_Q))
+        if heldout:
+            return out
+        out["K"] = rnd(_unit_rows(cfg, views, device, seed, _TID_K))
+        out["V"] = rnd(_normal_rows(cfg, views, device, seed, _TID_V))
+    else:
+        X = _latents(cfg, views, device, seed)
+        out["Q"] = rnd(_project(X, _projection(cfg, _TID_Q, device), True))
+        if heldout:
+            return out
+        out["K"] = rnd(_project(X, _projection(cfg, _TID_K, device), True))
+        out["V"] = rnd(_project(X, _projection(cfg, _TID_V, device), False))
+        del X
     C = cfg.heads * cfg.d
     out["conv_w"] = _randn((C, 3, 3), seed, _TID_CONV, 0, device) * (1.0 / 3.0)
     std = math.sqrt(2.0 / (cfg.d + cfg.h))

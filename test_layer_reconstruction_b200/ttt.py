@@ -24,8 +24,9 @@ __all__ = [
 OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
 EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
                     "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
-                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_grad", "ttt_sgd_update",
-                    "ttt_write_muon", "ttt_layer_muon", "ttt_grad_dot", "ttt_muon_update")
+                    "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_read_noalloc_status",
+                    "ttt_grad", "ttt_sgd_update", "ttt_write_muon", "ttt_layer_muon", "ttt_grad_dot",
+                    "ttt_muon_update")
 KERNEL_KINDS = 6
 
 
@@ -95,6 +96,8 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_status_str.restype = ctypes.c_char_p
     lib.ttt_read_noalloc.argtypes = [DP, P, P, P, P]
     lib.ttt_read_noalloc.restype = I
+    lib.ttt_read_noalloc_status.argtypes = [P]
+    lib.ttt_read_noalloc_status.restype = I
     lib.ttt_profile_start.argtypes = []
     lib.ttt_profile_stop.argtypes = [ctypes.POINTER(KernelTimes)]
     lib.ttt_kernel_name.argtypes = [I]

@@ -5,10 +5,11 @@ ttt_grad_dot / ttt_muon_update.
 Tolerances.  The Newton-Schulz step is checked against the oracle on the same
 gradient (FP32 iteration against float64: 1e-4 of the step).  The dot-product
 gradient has the mean-squared path's error (bf16 operands, FP32
-accumulation): 2e-2, as for the SGD update.  End to end, the oracle shows
-that NS5 magnifies an elementwise relative gradient perturbation about 3x on
-these gradients (1e-2 noise moves the step by 3.1e-2), so the Muon update is
-held to 3 x 2e-2 = 6e-2 of its size, and theta* and O to what that implies.
+accumulation): 2e-2, as for the SGD update.  The oracle shows that NS5
+magnifies an elementwise relative gradient perturbation about 3x on these
+gradients (1e-2 noise moves the step by 3.1e-2), so the Muon update itself
+is held to 3 x 2e-2 = 6e-2 of its size and theta* to what that implies; the
+read O is held to the layer's own 2e-2.
 """
 import numpy as np
 import pytest
@@ -17,7 +18,7 @@ import torch
 from oracle import ttt_oracle as orc
 from test_layer_reconstruction_b200 import inputs as tin
 from test_layer_reconstruction_b200 import sharded, ttt
-from ttt_testlib import TOL_DELTA, TOL_O, dims_of, normwise
+from ttt_testlib import TOL_DELTA, TOL_O, dims_of, normwise, report
 
 pytestmark = pytest.mark.gpu
 
@@ -94,13 +95,19 @@ def test_layer_muon_matches_oracle(name, heads):
     torch.cuda.synchronize()
     W = [t.double().numpy() for t in tin.unpack_theta(theta.cpu(), cfg.heads, cfg.d, cfg.h)]
     Og = O.double().cpu().numpy()
+    worst_d, worst_t, worst_o = 0.0, 0.0, 0.0
     for hd, (th0, th_ref, O_ref) in _oracle_muon(cfg, inp, 2, heads).items():
         for m in range(3):
             d_ref = th_ref[m] - th0[m]
-            assert normwise(W[m][hd] - th0[m], d_ref) <= TOL_MUON_DELTA, (hd, m)
+            e_d = normwise(W[m][hd] - th0[m], d_ref)
+            e_t = normwise(W[m][hd], th_ref[m])
+            worst_d, worst_t = max(worst_d, e_d), max(worst_t, e_t)
+            assert e_d <= TOL_MUON_DELTA, (hd, m)
             # theta* moves by at most the step's error
-            assert normwise(W[m][hd], th_ref[m]) <= TOL_MUON_DELTA * np.max(np.abs(d_ref)) / np.max(np.abs(th_ref[m]))
-        assert normwise(Og[:, hd], O_ref) <= max(TOL_O, TOL_MUON_DELTA), hd
+            assert e_t <= TOL_MUON_DELTA * np.max(np.abs(d_ref)) / np.max(np.abs(th_ref[m]))
+        worst_o = max(worst_o, normwise(Og[:, hd], O_ref))
+    report(f"muon_{name}", delta=worst_d, theta=worst_t, O=worst_o)
+    assert worst_o <= TOL_O, worst_o
 
 
 def test_muon_write_equals_its_pieces_bitwise():

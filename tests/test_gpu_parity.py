@@ -27,9 +27,9 @@ CONV_CASES = [
     _cfg(1, 1, 1, 0, 1, 32, 64),
     _cfg(2, 5, 7, 2, 16, 64, 256),
     _cfg(1, 2, 3, 5, 1, 64, 256),
-    _cfg(2, 41, 41, 1, 1, 32, 64),      # a 32-channel slab does not fit twice in shared memory: 16
-    _cfg(3, 37, 37, 5, 1, 16, 32),      # 16 channels in all: 16-channel slab
-    _cfg(2, 2, 300, 1, 1, 32, 64),      # grid wider than a TMA box: row kernel
+    _cfg(2, 41, 41, 1, 1, 32, 64),      # 41 rows: the last 3-row band is ragged (41 = 13 * 3 + 2)
+    _cfg(3, 37, 37, 5, 1, 16, 32),      # 16 channels: 4 threads per row, most of the block idle
+    _cfg(2, 2, 300, 1, 1, 32, 64),      # 300 columns: many passes of the 8-column shared-memory ring
 ]
 
 

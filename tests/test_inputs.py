@@ -1,7 +1,8 @@
 """The seeded input generator: shapes, value grid, normalisation, reproducibility
-of any view subset, and the token structure the draws are meant to carry
-(V at a token linearly predictable from K at that token, as for projections
-of one token feature)."""
+of any view subset, and the token structure of each family of draws: the
+workloads' own draws keep K, Q and V independent; the correlated family makes
+V at a token linearly predictable from K at that token, as for projections of
+one token feature."""
 import pytest
 import torch
 
@@ -15,6 +16,17 @@ def draw():
     return tin.make_inputs(SMALL)
 
 
+@pytest.fixture(scope="module")
+def draw_corr():
+    return tin.make_inputs(SMALL.with_draws("correlated"))
+
+
+def test_workloads_use_the_stated_draws():
+    assert all(c.draws == "stated" for c in tin.CONFIGS.values())
+    with pytest.raises(ValueError):
+        tin.make_inputs(SMALL.with_draws("other"))
+
+
 def test_shapes_and_parameter_scales(draw):
     c = SMALL
     assert draw["Q"].shape == draw["K"].shape == draw["V"].shape == (c.n, c.heads, c.d)
@@ -25,12 +37,27 @@ def test_shapes_and_parameter_scales(draw):
     assert abs(float(draw["conv_w"].std()) - 1.0 / 3.0) < 0.02
 
 
-def test_token_tensors_sit_on_the_bf16_grid_and_qk_rows_are_unit(draw):
-    for k in ("Q", "K", "V"):
-        assert torch.equal(draw[k], tin.bf16_round(draw[k]))
+def test_token_tensors_sit_on_the_bf16_grid_and_qk_rows_are_unit(draw, draw_corr):
+    for x in (draw, draw_corr):
+        for k in ("Q", "K", "V"):
+            assert torch.equal(x[k], tin.bf16_round(x[k]))
+        for k in ("Q", "K"):
+            norms = x[k].double().norm(dim=-1)
+            assert float((norms - 1).abs().max()) < 8e-3   # bf16 rounding of unit rows
+
+
+def test_stated_draws_are_standard_normal_directions_and_values(draw):
+    """K and Q rows are uniform directions (normalised N(0, I_d)): each entry has
+    mean 0 and variance 1/d; V is N(0, 1) elementwise."""
+    d = SMALL.d
     for k in ("Q", "K"):
-        norms = draw[k].double().norm(dim=-1)
-        assert float((norms - 1).abs().max()) < 8e-3   # bf16 rounding of unit rows
+        x = draw[k].double()
+        assert abs(float(x.mean())) < 0.01
+        assert abs(float(x.var()) * d - 1.0) < 0.03
+    v = draw["V"].double()
+    assert abs(float(v.mean())) < 0.01 and abs(float(v.std()) - 1.0) < 0.02
+    # fourth moment of a standard normal is 3
+    assert abs(float((v ** 4).mean()) - 3.0) < 0.1
 
 
 def test_fp32_draws_of_the_tiny_case_are_exactly_unit():
@@ -51,8 +78,17 @@ def test_view_subsets_and_permutations_reproduce_the_same_values(draw):
         assert torch.equal(again[k], draw[k])
 
 
-def test_heldout_views_have_new_latents_and_the_same_projections():
+def test_heldout_views_are_new_unit_rows():
     c = tin.CONFIGS["views2000_37x37p5_h1_d1024_h2048"].with_views(1)
+    main = tin.make_inputs(c)
+    held = tin.make_inputs(c, heldout=True, views=[0])
+    assert set(held) == {"Q"}
+    assert not torch.equal(held["Q"], main["Q"])
+    assert float((held["Q"].double().norm(dim=-1) - 1).abs().max()) < 8e-3
+
+
+def test_heldout_views_have_new_latents_and_the_same_projections():
+    c = tin.CONFIGS["views2000_37x37p5_h1_d1024_h2048"].with_views(1).with_draws("correlated")
     main = tin.make_inputs(c)
     held = tin.make_inputs(c, heldout=True, views=[0])
     assert set(held) == {"Q"}
@@ -61,13 +97,27 @@ def test_heldout_views_have_new_latents_and_the_same_projections():
     # so a least-squares map fitted from main Q to main K does not apply, but
     # re-drawing with the main seed reproduces the main Q exactly
     c2 = tin.LayerConfig(c.name, 1, c.grid_h, c.grid_w, c.n_special, c.heads, c.d, c.h, c.steps, c.lr, c.seed,
-                         heldout_views=1, heldout_seed=c.seed)
+                         heldout_views=1, heldout_seed=c.seed, draws="correlated")
     assert torch.equal(tin.make_inputs(c2, heldout=True)["Q"], main["Q"])
 
 
-def test_v_is_linearly_predictable_from_k_at_the_same_token(draw):
+def _r2(A, B):
+    sol = torch.linalg.lstsq(A, B).solution
+    return 1 - float(((A @ sol - B) ** 2).sum() / (B ** 2).sum())
+
+
+def test_stated_v_is_independent_of_k(draw):
+    """With independent draws a least-squares map from K (d regressors over
+    n tokens) explains only the chance fraction ~d/n of V."""
+    n, d = SMALL.n, SMALL.d
+    for hd in (0, SMALL.heads - 1):
+        assert _r2(draw["K"][:, hd].double(), draw["V"][:, hd].double()) < 3 * d / n
+
+
+def test_correlated_v_is_linearly_predictable_from_k_at_the_same_token(draw_corr):
     """V = x P_V and K = x P_K / |x P_K|: a linear map from K explains most of V
     (up to the per-row scale |x P_K|); shuffling the tokens destroys it."""
+    draw = draw_corr
     g = torch.Generator().manual_seed(0)
     for hd in (0, SMALL.heads - 1):
         A = draw["K"][:, hd].double()

@@ -5,8 +5,11 @@ allocations, or all device memory already handed to a pool the caller does
 not control).  For them the library offers a read whose scratch is a fixed
 array inside the library.  This test calls it through the C ABI twice in a
 row and checks each result against ttt_read with a caller-allocated
-workspace, and checks that oversized shapes are refused.  It lives in its own
-file, collected last, and passes alone or after the other tests.
+workspace, reads the call's device status through ttt_read_noalloc_status
+after each call, checks that the second call allocates no device memory
+through the caller's allocator, and checks that shapes beyond the fixed
+scratch are refused before anything runs.  It lives in its own file,
+collected last, and passes alone or after the other tests.
 """
 import ctypes
 
@@ -20,11 +23,14 @@ from ttt_testlib import TOL_O, bf16_inputs, normwise, to_device
 pytestmark = pytest.mark.gpu
 
 
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
 def _noalloc(lib, cfg, Q, theta, O):
     dm = ttt.Dims.of(cfg)
     return lib.ttt_read_noalloc(ctypes.byref(dm), ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(theta.data_ptr()),
-                                ctypes.c_void_p(O.data_ptr()),
-                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+                                ctypes.c_void_p(O.data_ptr()), _stream())
 
 
 def test_read_noalloc_matches_read_twice():
@@ -35,10 +41,15 @@ def test_read_noalloc_matches_read_twice():
         inp = bf16_inputs(tin.make_inputs(cfg))
         dev = to_device(inp)
         ref = ttt.read(dev["Q"], dev["theta"], cfg).float().cpu().numpy()
-        for _ in range(2):
-            O = torch.full_like(dev["Q"], float("nan"))
+        outs = [torch.full_like(dev["Q"], float("nan")) for _ in range(2)]
+        torch.cuda.synchronize()
+        for i, O in enumerate(outs):
+            before = torch.cuda.memory_allocated()
             assert _noalloc(lib, cfg, dev["Q"], dev["theta"], O) == 0
-            torch.cuda.synchronize()
+            assert lib.ttt_read_noalloc_status(_stream()) == 0
+            if i == 1:
+                # the first call on a device may set up the array's address; later ones allocate nothing
+                assert torch.cuda.memory_allocated() == before
             got = O.float().cpu().numpy()
             assert normwise(got, ref) <= TOL_O
 
@@ -51,3 +62,4 @@ def test_read_noalloc_rejects_shapes_beyond_its_scratch():
     theta = torch.zeros(3 * cfg.heads * cfg.d * cfg.h, dtype=torch.float32, device="cuda")
     O = torch.empty_like(Q)
     assert _noalloc(lib, cfg, Q, theta, O) == -4
+    assert lib.ttt_read_noalloc_status(_stream()) == 0

@@ -4,8 +4,21 @@ Tolerance reading (norm-wise "max relative error"): err(a, ref) =
 max|a - ref| / max|ref|, per tensor and per head.  The GPU path must meet
 O <= 2e-2 and theta* <= 1e-2; the stricter diagnostic on the update itself,
 delta = theta* - theta0, must meet <= 2e-2.
+
+theta* is returned in float32, and each step rounds theta to it: the stored
+theta* differs from the exact theta_t - lr * g by up to half an ulp of
+|theta| per step, whatever the arithmetic before it.  At the workloads' step
+sizes one step moves theta by ~1e-6 while half an ulp of |theta| ~ 0.3 is
+1.5e-8, so that resolution alone is a few percent of delta on the largest
+workloads.  The delta diagnostic is therefore measured beyond it:
+    (max|delta_gpu - delta_ref| - steps * ulp32(max|theta|) / 2) / max|delta_ref|.
+The gradient itself (``ttt_grad``, float32 with no theta added) carries no
+such term and is compared plainly.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -67,8 +80,29 @@ def oracle_layer(cfg: tin.LayerConfig, inp, heads=None, steps=None, lr=None):
     return res
 
 
-def compare_theta(cfg, inp, theta_gpu: torch.Tensor, ref, heads=None):
-    """Return worst (theta err, delta err) over heads and the three matrices."""
+def f32_resolution(theta_max: float, steps: int) -> float:
+    """Largest error that rounding theta to float32 after each of `steps`
+    steps can leave on theta*: half an ulp of the largest |theta| per step."""
+    if theta_max <= 0 or steps <= 0:
+        return 0.0
+    ulp = 2.0 ** (np.floor(np.log2(theta_max)) - 23)
+    return steps * 0.5 * float(ulp)
+
+
+def delta_error(g, r, t0, steps) -> float:
+    """Norm-wise error of delta = theta* - theta0 beyond the float32 resolution of theta*."""
+    g, r, t0 = (np.asarray(x, np.float64) for x in (g, r, t0))
+    dr = r - t0
+    den = np.max(np.abs(dr))
+    q = f32_resolution(max(np.max(np.abs(r)), np.max(np.abs(t0))), steps)
+    num = max(0.0, float(np.max(np.abs((g - t0) - dr))) - q)
+    return num / den if den > 0 else num
+
+
+def compare_theta(cfg, inp, theta_gpu: torch.Tensor, ref, heads=None, steps=None):
+    """Return worst (theta err, delta err) over heads and the three matrices;
+    the delta error is measured beyond the float32 resolution of theta*."""
+    steps = cfg.steps if steps is None else steps
     W1g, W3g, W2g = tin.unpack_theta(theta_gpu.detach().cpu(), cfg.heads, cfg.d, cfg.h)
     gpu = {"W1": W1g, "W3": W3g, "W2": W2g}
     heads = list(ref["W1"].keys()) if heads is None else heads
@@ -79,7 +113,7 @@ def compare_theta(cfg, inp, theta_gpu: torch.Tensor, ref, heads=None):
             r = ref[name][hd]
             t0 = inp[name][hd].double().numpy()
             worst_t = max(worst_t, normwise(g, r))
-            worst_d = max(worst_d, normwise(g - t0, r - t0))
+            worst_d = max(worst_d, delta_error(g, r, t0, steps))
     return worst_t, worst_d
 
 
@@ -117,3 +151,25 @@ def guards_intact(buf) -> bool:
     """True when both canary bands of a `guarded` buffer are untouched."""
     b = buf.cpu()
     return bool((b[:GUARD] == CANARY).all()) and bool((b[-GUARD:] == CANARY).all())
+
+
+def report(test: str, **values) -> None:
+    """Append the measured errors of a parity test as one JSON line to the file
+    named by TTT_PARITY_REPORT (nothing when it is unset)."""
+    path = os.environ.get("TTT_PARITY_REPORT")
+    if not path:
+        return
+    with open(path, "a") as f:
+        f.write(json.dumps({"test": test, **{k: (float(v) if isinstance(v, (float, np.floating)) else v)
+                                              for k, v in values.items()}}) + "\n")
+
+
+def oracle_grad_sum(K, Vp, th0, chunk=None):
+    """d/dtheta of (1/2) sum_i ||T(k_i) - v'_i||^2 by the oracle (one head), the
+    quantity ttt_grad returns: n/2 times the gradient of the mean-squared loss."""
+    n = K.shape[0]
+    if chunk is None or chunk >= n:
+        g = orc.mse_grad(K, Vp, *th0)
+    else:
+        g = orc.mse_grad_chunked(K, Vp, *th0, chunk=chunk)
+    return tuple(x * (n / 2.0) for x in g)
