@@ -203,20 +203,63 @@ def run_reference(args, cfg):
     return 0
 
 
-def _kernel_work(cfg):
-    """Algorithmic work of one launch of each kernel kind (bytes or FLOPs)."""
-    n, H, d, h = cfg.n, cfg.heads, cfg.d, cfg.h
+def _kernel_work(cfg, n_read=None):
+    """Algorithmic work of each kernel kind in ONE step (a layer call, plus the
+    held-out read where the workload has one): bytes for the HBM-bound kinds,
+    FLOPs for the tensor-core ones.  `n_read` is the number of tokens read
+    (the layer's Q plus held-out queries)."""
+    n, H, d, h, st = cfg.n, cfg.heads, cfg.d, cfg.h, cfg.steps
+    n_read = n if n_read is None else n_read
     tok = n * H * d * 2
+    theta = 3 * H * d * h * 4
+    hidp = 128 * math.ceil(h / 128)
     return {
-        "shortconv2d": ("hbm", 2 * tok + H * d * 9 * 4),             # read V, write V'
-        "swiglu_fwd_residual": ("tensor", 6.0 * d * h * n * H),      # Z1, Z3, Y
-        "swiglu_bwd_partials": ("tensor", 8.0 * d * h * n * H),      # dA, dW1, dW3, dW2
-        "swiglu_fwd_read": ("tensor", 6.0 * d * h * n * H),
-        # read theta (f32); write the W1|W3 bf16 image and the bf16 and f16 W2 images
-        "pack_theta": ("hbm", 3 * H * d * h * 4 + 4 * H * 128 * math.ceil(h / 128) * d * 2),
+        "shortconv2d": ("hbm", 2 * tok + H * d * 9 * 4),                 # read V, write V'
+        "swiglu_fwd_residual": ("tensor", st * 6.0 * d * h * n * H),     # Z1, Z3, Y
+        "swiglu_bwd_partials": ("tensor", st * 8.0 * d * h * n * H),     # dA, dW1, dW3, dW2
+        "swiglu_fwd_read": ("tensor", 6.0 * d * h * n_read * H),
+        # read theta (f32); write the operand images (bf16 W1|W3, bf16 and f16 W2)
+        "pack_theta": ("hbm", (st + 1) * (theta + 4 * H * hidp * d * 2)),
         # read theta, write theta* (the split-K partials it also reads are a by-product of the tiling)
-        "reduce_sgd": ("hbm", 2 * 3 * H * d * h * 4),
+        "reduce_sgd": ("hbm", st * 2 * theta),
+        # the tensor-core GEMMs of the wide-head path and the surround
+        "gemm_gate": ("tensor", 4.0 * d * h * H * (st * n + n_read)),     # Z1, Z3
+        "gemm_residual": ("tensor", st * 2.0 * d * h * n * H),            # Y = A W2
+        "gemm_dz": ("tensor", st * 2.0 * d * h * n * H),                  # dA = E W2^T
+        "gemm_wgrad": ("tensor", st * 6.0 * d * h * n * H),               # dW1, dW3, dW2
+        "gemm_store": ("tensor", 2.0 * d * h * n_read * H),               # O = A W2
+        "gemm_qkv_l2norm": ("tensor", 3 * 2.0 * n * (H * d) ** 2),        # X Wq, X Wk, X Wv
     }
+
+
+def _kernel_table(prof, work, steps, peaks):
+    """Per kernel kind: launches and time per step, achieved rate on its
+    algorithmic work per step, fraction of the measured peak."""
+    total = sum(r["total_ms"] for k, r in prof.items() if not k.startswith("_"))
+    kernels = {}
+    for name, rec in prof.items():
+        if name.startswith("_") or rec["launches"] == 0 or name not in work:
+            continue
+        bound, amount = work[name]
+        ms_step = rec["total_ms"] / steps
+        extra = {}
+        if bound == "tensor":
+            # each launch is timed on its own (CUDA events around every launch), so the
+            # burst GEMM peak is the denominator; the sustained figure is a second number
+            achieved = amount / (ms_step / 1e3) / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+            extra = {"peak_sustained": peaks["bf16_tflops_sustained"],
+                     "frac_sustained": achieved / peaks["bf16_tflops_sustained"]}
+        else:
+            achieved = amount / (ms_step / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        kernels[name] = {"launches_per_step": rec["launches"] / steps,
+                         "ms_per_launch": rec["total_ms"] / rec["launches"], "ms_per_step": ms_step,
+                         "share": rec["total_ms"] / max(1e-9, total), "bound": bound, "achieved": achieved,
+                         "peak": peak, "unit": unit, "frac": achieved / peak if peak else None, **extra}
+    return kernels
 
 
 def run_ours(args, cfg):
@@ -275,8 +318,21 @@ def run_ours(args, cfg):
         def layer_call(Q_, K_, V_, w_, th0_):
             return ttt.layer(Q_, K_, V_, w_, th0_, cfg.lr, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
 
+    # Workloads with held-out views: each step also reads their queries with
+    # the frozen theta* (the localisation-style query path).
+    n_read = cfg.n
+    held = None
+    if cfg.heldout_views > 0:
+        hcfg = cfg.with_views(cfg.heldout_views)
+        Qh = tin.make_inputs(cfg, device="cuda", heldout=True)["Q"].to(torch.bfloat16).contiguous()
+        held = (hcfg, Qh, torch.empty_like(Qh), ttt.make_workspace(hcfg, ttt.OP_READ))
+        n_read += hcfg.n
+
     def step():
-        layer_call(Q, K, V, conv_w, theta0)
+        th_, _ = layer_call(Q, K, V, conv_w, theta0)
+        if held is not None:
+            hcfg_, Qh_, Oh_, wsr_ = held
+            ttt.read(Qh_, th_, hcfg_, O=Oh_, workspace=wsr_)
 
     for _ in range(args.warmup):
         step()
@@ -307,32 +363,8 @@ def run_ours(args, cfg):
 
     # per-kernel roofline from the live event timings
     peaks = _peaks()
-    work = _kernel_work(cfg)
-    kernels = {}
-    for name, rec in prof.items():
-        if name.startswith("_") or rec["launches"] == 0:
-            continue
-        bound, amount = work[name]
-        per_launch_ms = rec["total_ms"] / rec["launches"]
-        extra = {}
-        if bound == "tensor":
-            # each kernel is timed on its own (CUDA events around every launch), so the
-            # burst GEMM peak is the denominator; the sustained figure is a second number
-            achieved = amount / (per_launch_ms / 1e3) / 1e12
-            peak = peaks["bf16_tflops"]
-            unit = "TFLOP/s"
-            extra = {"peak_sustained": peaks["bf16_tflops_sustained"],
-                     "frac_sustained": achieved / peaks["bf16_tflops_sustained"]}
-        else:
-            achieved = amount / (per_launch_ms / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            unit = "GB/s"
-        kernels[name] = {"launches_per_step": rec["launches"] / args.steps, "ms_per_launch": per_launch_ms,
-                         "share": rec["total_ms"] / max(1e-9, sum(r["total_ms"] for k, r in prof.items()
-                                                                  if not k.startswith("_"))),
-                         "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak if peak else None, **extra}
-    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches_per_step"])
+    kernels = _kernel_table(prof, _kernel_work(cfg, n_read), args.steps, peaks)
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     dk = kernels[dom]
     traffic = _traffic_from_profiles(dom, cfg.name)
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
@@ -407,7 +439,7 @@ def run_ours(args, cfg):
     # are contiguous token ranges) and the write-only / read-only split at 100
     # views, each timed with CUDA events like the main run.
     sweep, paths = None, None
-    if rank == 0 and world == 1 and not args.no_sweep:
+    if rank == 0 and world == 1 and not args.no_sweep and cfg.name == DEFAULT_CONFIG:
         T = cfg.tokens_per_view
 
         def time_calls(fn, reps=3, warm=2):
@@ -481,6 +513,30 @@ def run_ours(args, cfg):
             "tokens_per_s": cfg.n / (ms_st / 1e3),
             "host_bytes_per_call": int((cfg.steps * 2 + 2) * hq.numel() * 2)}
         del hq, hk, hv
+    if rank == 0 and world == 1 and not args.no_sweep and cfg.name == DEFAULT_CONFIG and not args.no_surround:
+        # The layer's surround on the same workload: q = L2(X Wq), k = L2(X Wk),
+        # v = X Wv (one GEMM launch, the normalisation in its epilogue), the
+        # layer, out = O Wo.
+        sx = tin.make_surround(cfg, device="cuda")
+        sdev = {k: sx[k].to(torch.bfloat16).contiguous() for k in ("X", "Wq", "Wk", "Wv", "Wo")}
+        del sx
+        torch.cuda.empty_cache()
+        ws_a = ttt.make_workspace(cfg, ttt.OP_ATTENTION)
+        s_out = torch.empty_like(sdev["X"])
+        ttt.profile_start()
+        ms_att = time_calls(lambda: ttt.attention(sdev["X"], sdev["Wq"], sdev["Wk"], sdev["Wv"], sdev["Wo"], conv_w,
+                                                  theta0, cfg.lr, cfg.steps, cfg, theta_out=theta, out=s_out,
+                                                  workspace=ws_a))
+        prof_att = ttt.profile_stop()
+        if ttt.check_status(ws_a) != 0:
+            raise SystemExit("device status word set during the attention layer")
+        work_att = _kernel_work(cfg)
+        work_att["gemm_store"] = ("tensor", 2.0 * cfg.n * (cfg.heads * cfg.d) ** 2)   # out = O Wo
+        tab = _kernel_table(prof_att, work_att, calls, _peaks())
+        paths["attention_surround"] = {
+            "views": cfg.n_views, "ms_per_call": round(ms_att, 3), "tokens_per_s": cfg.n / (ms_att / 1e3),
+            "qkv_projection": tab.get("gemm_qkv_l2norm"), "output_projection": tab.get("gemm_store")}
+        del sdev, s_out, ws_a
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -497,7 +553,10 @@ def run_ours(args, cfg):
                        "l2": f"no flush: every token tensor ({cfg.n * cfg.heads * cfg.d * 2 / 1e9:.2f} GB) exceeds the 126 MB L2",
                        "parallelism": (f"{world} GPUs: one {cfg.n_views * world}-view collection sharded by views "
                                        f"({cfg.n_views} per GPU), gradient all-gather per step (NCCL)" if shard
-                                       else f"{world} independent replicas" if world > 1 else "1 GPU")},
+                                       else f"{world} independent replicas" if world > 1 else "1 GPU"),
+                       **({"heldout_views": cfg.heldout_views, "tokens_read": n_read,
+                           "value_counts": "the layer's tokens (the held-out read is extra work in each step)"}
+                          if cfg.heldout_views else {})},
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": gpu_launches, "clocks": clk, "sweep": sweep, "paths": paths,
         }
@@ -548,6 +607,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the view-count sweep and write/read split")
+    ap.add_argument("--no-surround", action="store_true", help="skip the attention-surround measurement")
     ap.add_argument("--replicas", action="store_true",
                     help="with N > 1: independent scenes per GPU instead of one collection sharded by views")
     ap.add_argument("--shard", action="store_true",

@@ -41,11 +41,10 @@
  *   d in {16, 32, 64} and 1 <= h <= 256 (padded internally to a multiple of
  *   128 with zero weights, which is exact): the fused tensor-core kernels; or
  *   d and h multiples of 64 (d <= 8192, h <= 32768), e.g. d = 1024, h = 2048:
- *   the wide-head path, which runs the products as bf16 cuBLAS GEMMs with FP32
- *   accumulation over chunks of 131072 tokens.  Its first call on a device
- *   creates that device's cuBLAS handle (cuBLAS allocates its own small state
- *   then); the GEMMs use the workspace for their scratch.  Calls of the wide
- *   path on one device are serialised while they enqueue.
+ *   the wide-head path, which runs the products as the library's own bf16
+ *   tensor-core GEMMs (FP32 accumulation, the gate, residual and chain rule
+ *   fused into their epilogues) over chunks of 262144 tokens, the weight
+ *   gradients summed over the chunks in a fixed order.
  * Other shapes return TTT_EUNSUPPORTED.
  */
 #ifndef TTT_H_
@@ -82,8 +81,14 @@ typedef enum ttt_op {
   TTT_OP_WRITE = 0,       /* ttt_write                                         */
   TTT_OP_READ = 1,        /* ttt_read                                          */
   TTT_OP_LAYER = 2,       /* ttt_layer                                         */
-  TTT_OP_LAYER_HOST = 3   /* ttt_layer_host: also holds device copies of Q,K,V,conv_w,theta,O */
+  TTT_OP_LAYER_HOST = 3,  /* ttt_layer_host: also holds device copies of Q,K,V,conv_w,theta,O */
+  TTT_OP_ATTENTION = 4    /* ttt_attention: the layer plus q, k, v and O of the surround */
 } ttt_op;
+
+typedef enum ttt_inner {
+  TTT_INNER_SGD = 0,      /* mean-squared loss, SGD steps (ttt_layer)              */
+  TTT_INNER_MUON = 1      /* dot-product loss, Muon steps (ttt_layer_muon)         */
+} ttt_inner;
 
 /* Bytes of device workspace an op needs for these dims; 0 if dims are invalid
  * or unsupported. */
@@ -176,6 +181,40 @@ int ttt_layer(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const 
               float* theta_out, uint16_t* O, void* workspace, size_t workspace_bytes,
               void* stream);
 
+/* The global attention layer with the TTT layer in place of softmax
+ * attention (VGG-T^3 summary, Sec. 3 "QKV projection with normalization",
+ * Eq. 1, with LN_q and LN_k replaced by L2 normalisation as in "The LayerNorm
+ * removal"; then the output projection):
+ *   q = L2(X Wq), k = L2(X Wk)  each (token, head) row of d scaled to unit
+ *                               norm (a zero row stays zero),
+ *   v = X Wv                    one tensor-core GEMM launch for all three, the
+ *                               normalisation in its epilogue, q, k, v rounded
+ *                               to bf16 once;
+ *   the layer on (q, k, v)      inner = TTT_INNER_SGD: as ttt_layer;
+ *                               TTT_INNER_MUON: as ttt_layer_muon;
+ *   out = O Wo                  a tensor-core GEMM, bf16 output.
+ * X, out: bf16 [n][C] with C = heads * d; Wq, Wk, Wv, Wo: bf16 [C][C] in the
+ * row-vector form x W (no biases); conv_w, theta0, theta_out as for
+ * ttt_layer.  Requires d = 64 and h <= 256 (the fused layer kernels); other
+ * shapes return TTT_EUNSUPPORTED.  Workspace:
+ * ttt_workspace_bytes(dims, TTT_OP_ATTENTION). */
+int ttt_attention(const ttt_dims* dims, const uint16_t* X, const uint16_t* Wq, const uint16_t* Wk,
+                  const uint16_t* Wv, const uint16_t* Wo, const float* conv_w, const float* theta0,
+                  float lr, int steps, int inner, float* theta_out, uint16_t* out,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* C = A B on the library's tensor-core GEMM (the kernel of the projections
+ * and of the wide-head path): bf16 operands, FP32 accumulation, bf16 output
+ * rounded to nearest even.  A is M x K, stored row-major as [M][lda]
+ * (a_layout 0) or as its transpose [K][lda] (a_layout 1); B is K x N, stored
+ * as [K][ldb] (b_layout 0) or as its transpose [N][ldb] (b_layout 1, a linear
+ * layer's [out][in] weight); C is [M][ldc].  M, N, K >= 1; N and the three
+ * leading dimensions multiples of 8 elements; pointers 16-byte aligned (else
+ * TTT_EALIGN).  Needs no workspace. */
+int ttt_gemm_bf16(int M, int N, int K, const uint16_t* A, int64_t lda, int a_layout,
+                  const uint16_t* B, int64_t ldb, int b_layout, uint16_t* C, int64_t ldc,
+                  void* stream);
+
 /* ttt_layer on HOST buffers: copies Q, K, V, conv_w, theta0 to device copies
  * inside the workspace, runs the layer, and copies theta* and O back to the
  * host buffers.  On the fused path the copies are pipelined: conv_w, theta0,
@@ -227,6 +266,16 @@ int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta
  * may be used again in the process. */
 int ttt_read_noalloc_status(void* stream);
 
+/* Sets the limit, in SM clocks, of every bounded wait in the tensor-core
+ * kernels launched after the call (process-wide); 0 (the default) selects the
+ * built-in limit of 4e9 clocks (about two seconds).  A wait that runs out
+ * makes its kernel record TTT_EDEVICE in the status word, stop every role,
+ * let its copies and MMAs in flight finish, release its tensor memory and
+ * return, so the context stays usable.  For tests of that path: a limit of a
+ * few hundred clocks makes waits run out on any workload.  Returns TTT_OK, or
+ * TTT_EINVAL for a negative limit. */
+int ttt_set_wait_limit(long long clocks);
+
 /* Synchronises `stream`, then reads the device status word of `workspace`:
  * TTT_OK, TTT_EDEVICE if a kernel recorded a fault (the word is cleared), or
  * TTT_ECUDA. */
@@ -245,7 +294,7 @@ const char* ttt_status_str(int status);
  * The "reduce_sgd" kind covers every theta-sized step kernel: the split-K
  * reduction with its SGD step, the fixed-order update of ttt_sgd_update and
  * the Newton-Schulz step of the Muon entry points. */
-#define TTT_KERNEL_KINDS 6
+#define TTT_KERNEL_KINDS 12
 typedef struct ttt_kernel_times {
   int32_t launches[TTT_KERNEL_KINDS];
   float total_ms[TTT_KERNEL_KINDS];

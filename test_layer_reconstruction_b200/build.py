@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libttt.so")
 SOURCES = ["ttt_capi.cu"]
-HEADERS = ["sm100.cuh", "fwd.cuh", "bwd.cuh", "update.cuh", "conv.cuh", "wide.cuh"]
+HEADERS = ["sm100.cuh", "fwd.cuh", "bwd.cuh", "update.cuh", "conv.cuh", "gemm.cuh", "wide.cuh"]
 
 
 def nvcc() -> str:
@@ -43,7 +43,6 @@ def build(force: bool = False, verbose: bool = False, out: str = None, defines=(
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
-    cmd += ["-lcublas"]   # library GEMMs of the wide-head path
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)

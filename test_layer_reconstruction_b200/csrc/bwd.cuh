@@ -63,6 +63,7 @@ struct BwdParams {
   int n, heads, units, slices;   // units = ceil(n / kUnit); slices = HIDP / 128
   int max_contrib;
   unsigned int* status;
+  long long wait_clocks;         // limit of a bounded wait (<= 0: the default)
 };
 
 template <int D>
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const Abort ab{abort_flag, p.status};
+  const Abort ab{abort_flag, p.status, p.wait_clocks};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // CTAs come in groups of `slices`: CTA group*slices + s handles hidden slice s
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // moves matrix g (2 dW1^T, dW3^T, dW2), row = hidden unit.
     auto dump = [&](long long pair) -> bool {
       TTT_TR_LAP(0);
-      if (!mbar_wait(&bars[BB_ACC_FULL], dumps & 1, ab)) return false;
+      if (!mbar_wait_warp(&bars[BB_ACC_FULL], dumps & 1, ab)) return false;
       TTT_TR_LAP(5);
       tc_fence_after();
       const long long first_item = (pair / p.slices) * static_cast<long long>(p.units);
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // warpgroups 1 and 2 the W3^T and W2 rows into shared memory (the K-major,
     // swizzled A operands of Z3^T and dA^T).
     auto load_weights = [&](int head) -> bool {
-      if (seg > 0 && !mbar_wait(&bars[BB_W_EMPTY], (seg - 1) & 1, ab)) return false;
+      if (seg > 0 && !mbar_wait_warp(&bars[BB_W_EMPTY], (seg - 1) & 1, ab)) return false;
       tc_fence_after();
       const size_t hidp = static_cast<size_t>(p.slices) * 128;
       const uint4* src = reinterpret_cast<const uint4*>(
@@ -401,7 +402,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const uint32_t pa = j & 1;
       TTT_TR_LAP(0);
-      if (!(ok = mbar_wait(&bars[BB_FULL + ub], uph, ab))) break;
+      if (!(ok = mbar_wait_warp(&bars[BB_FULL + ub], uph, ab))) break;
       TTT_TR_LAP(1);
       tc_fence_after();
       uint32_t zu[16], z3[16], da[16];
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // its slot once the dW MMAs of unit j-2 have read it.
       tmem_st8(tu, pz1);
       tmem_st8(tu + 8, pz3);
-      if (!(ok = mbar_wait(&bars[BB_PA_EMPTY + pa], ((j >> 1) & 1) ^ 1, ab))) break;
+      if (!(ok = mbar_wait_warp(&bars[BB_PA_EMPTY + pa], ((j >> 1) & 1) ^ 1, ab))) break;
       TTT_TR_LAP(4);
       tc_fence_after();
       tmem_st8(tbase + L::cPA + pa * 24 + 8 * g + lane_off, pav);

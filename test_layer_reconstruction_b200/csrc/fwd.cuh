@@ -45,6 +45,7 @@ struct FwdParams {
   __nv_bfloat16* out;            // [n][heads][D]
   int n, heads, tiles;
   unsigned int* status;
+  long long wait_clocks;         // limit of a bounded wait (<= 0: the default)
 };
 
 template <int D, int HIDP>
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const Abort ab{abort_flag, p.status};
+  const Abort ab{abort_flag, p.status, p.wait_clocks};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const long long total = static_cast<long long>(p.heads) * p.tiles;
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_x);
       if (WRITE) tma_prefetch_desc(&tm_vp);
       int cur_head = -1;
-      uint32_t wl = 0, j = 0;
+      uint32_t wl = 0, j = 0, nx = 0, nvp = 0;
       Cursor pf;
       pf.init(it0, p.tiles);
       for (int k = 0; k < kPrefetchAhead && pf.it < it1; ++k, pf.next(p.tiles)) {
@@ -219,22 +220,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         TTT_TR_LAP(1);
         mbar_arrive_expect_tx(&bars[FB_X_FULL + s], L::kTile);
         tma_load_2d(smem + L::off_x + s * L::kTile, &tm_x, &bars[FB_X_FULL + s], head * D, tile * kTileM);
+        ++nx;
         if (WRITE) {
           TTT_TR_LAP(0);
           if (!mbar_wait(&bars[FB_VP_EMPTY + s], ph ^ 1, ab)) break;
           TTT_TR_LAP(2);
           mbar_arrive_expect_tx(&bars[FB_VP_FULL + s], L::kTile);
           tma_load_2d(smem + L::off_vp + s * L::kTile, &tm_vp, &bars[FB_VP_FULL + s], head * D, tile * kTileM);
+          ++nvp;
         }
       }
       TTT_TR_LAP(0);
       TTT_TR_DUMP(WRITE ? 0 : 1);
-      // Drain: the last load issued into each barrier has landed before exit.
+      // Drain: the last load issued into each barrier has landed before exit
+      // (after an abort the X load of an item may have gone out without its V').
       if (wl > 0) mbar_drain(&bars[FB_W_FULL], (wl - 1) & 1);
-      for (uint32_t jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj) {
-        mbar_drain(&bars[FB_X_FULL + (jj & 1)], (jj >> 1) & 1);
-        if (WRITE) mbar_drain(&bars[FB_VP_FULL + (jj & 1)], (jj >> 1) & 1);
-      }
+      for (uint32_t jj = (nx >= 2 ? nx - 2 : 0); jj < nx; ++jj) mbar_drain(&bars[FB_X_FULL + (jj & 1)], (jj >> 1) & 1);
+      for (uint32_t jj = (nvp >= 2 ? nvp - 2 : 0); jj < nvp; ++jj)
+        mbar_drain(&bars[FB_VP_FULL + (jj & 1)], (jj >> 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ Z issuer
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto y_epilogue = [&](uint32_t jj, int head, int tile) -> bool {
       const uint32_t ys = jj & 1;
       TTT_TR_LAP(0);
-      if (!mbar_wait(&bars[FB_Y_FULL + ys], (jj >> 1) & 1, ab)) return false;
+      if (!mbar_wait_warp(&bars[FB_Y_FULL + ys], (jj >> 1) & 1, ab)) return false;
       TTT_TR_LAP(5);
       tc_fence_after();
       float y[kYHalf];
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[FB_Y_EMPTY + ys]);
       if (WRITE) {
-        if (!mbar_wait(&bars[FB_VP_FULL + ys], (jj >> 1) & 1, ab)) return false;
+        if (!mbar_wait_warp(&bars[FB_VP_FULL + ys], (jj >> 1) & 1, ab)) return false;
         const uint32_t vb = smem_u32(smem + L::off_vp + ys * L::kTile);
 #pragma unroll
         for (int ch = 0; ch < kYHalf / 8; ++ch) {
@@ -402,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; cu.it < it1 && ok; cu.next(p.tiles), ++j) {
       for (int c = pr; c < NC; c += 2, ++u) {
         TTT_TR_LAP(0);
-        if (!(ok = mbar_wait(&bars[FB_Z_FULL + pr], u & 1, ab))) break;
+        if (!(ok = mbar_wait_warp(&bars[FB_Z_FULL + pr], u & 1, ab))) break;
         TTT_TR_LAP(1);
         tc_fence_after();
         // Z slot columns: [Z1 (32) | Z3 (32)] of hidden 64c + 0..31, then of 64c + 32..63;
@@ -425,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + pr]);
         TTT_TR_LAP(2);
-        if (!(ok = mbar_wait(&bars[FB_A_EMPTY + pr], (u & 1) ^ 1, ab))) break;
+        if (!(ok = mbar_wait_warp(&bars[FB_A_EMPTY + pr], (u & 1) ^ 1, ab))) break;
         TTT_TR_LAP(3);
         tc_fence_after();
         tmem_st16(tg + pr * 32 + hf * 16 + lane_off, gk);

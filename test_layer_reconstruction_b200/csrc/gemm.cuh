@@ -1,0 +1,467 @@
+// gemm.cuh — persistent bf16 GEMM on the 5th-generation tensor cores with
+// fused epilogues, for the products that are plain dense GEMMs:
+//   * the wide-head layer (one head with d = 1024, h = 2048; VGG-T$^3$:
+//     Offline Feed-Forward 3D Reconstruction at Scale, Sec. 3.4, Eq. 3-5),
+//     where one head's fast weights no longer fit on chip, and
+//   * the layer's surround: the QKV projection with the per-head L2
+//     normalisation of q and k in its epilogue (Sec. 3, Eq. 1, and "The
+//     LayerNorm removal"), and the output projection.
+//
+// C[m][n] = sum_k A[m][k] B[k][n] with bf16 operands and FP32 accumulation
+// in tensor memory.  Each operand is read by TMA from a 2-D bf16 tensor in
+// one of two layouts:
+//   K-major : the operand's rows are M (or N) and K is contiguous (A stored
+//             [M][K], B stored [N][K]); TMA box 64 (K) x 128 rows.
+//   MN-major: the rows are K and M (or N) is contiguous (A stored [K][M],
+//             B stored [K][N]); TMA box 64 (M or N) x 64 (K rows).
+// Both use the 128-byte swizzle.  Tiles are 128 x 256 (M x N) with K steps
+// of 64: per stage one or two A boxes (16 KiB) and two or four B boxes
+// (32 KiB), four stages.  Each k step issues four M=128, N=256, K=16 MMAs;
+// at that shape an SS MMA reads 96 B/clk of shared memory, under the ~128
+// B/clk the tensor core takes, so it runs at full rate.
+//
+// One persistent CTA per SM walks the work items (problem, M tile, N tile,
+// K split) of up to three problems with a static stride.  Warp roles:
+//   warp 0     TMA producer
+//   warp 1     TMEM allocator and MMA issuer (warp-uniform, one elected lane)
+//   warps 4-11 epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (rows of
+//              the tile); warps 4-7 take the first half of the tile's
+//              columns, warps 8-11 the second.
+// The accumulator is double buffered in TMEM (2 x 256 columns), so the
+// epilogue of one tile overlaps the MMAs of the next.  Rows and columns past
+// a problem's M and N are computed on TMA's zero fill and not stored.
+//
+// Epilogues (template parameter):
+//   kEpiStore    out = bf16(C) (a column offset lets a tile land inside a
+//                wider row, e.g. one head's columns of [n][heads*d]).
+//   kEpiResidual out = bf16(C - R) with R a bf16 tensor of out's shape.
+//   kEpiL2Heads  the tile's columns are heads of 64: columns below
+//                `norm_cols` are divided by the L2 norm of their 64-column
+//                row segment (a zero segment stays zero), then bf16.
+//   kEpiGate     the tile's columns are [Z1 of 128 hidden units | Z3 of the
+//                same units]: A = silu(Z1) Z3, F1 = Z3 s (1 + Z1 (1 - s)) and
+//                F3 = silu(Z1) with s = sigmoid(Z1), each bf16 [rows][hidden]
+//                (F1 and F3 optional): A feeds the next products, and
+//                dZ1 = dA F1, dZ3 = dA F3 is the chain rule of the backward.
+//   kEpiDz       C = dA (columns = hidden units): dZ1 = dA F1, dZ3 = dA F3
+//                written in place over F1 and F3.
+//   kEpiAccF32   f32 [M][N] at out + split * split_stride = C, or += C when
+//                `accumulate`: the split-K partial sums of the weight
+//                gradients, each element owned by one CTA per launch, so the
+//                sums are deterministic.
+#pragma once
+#include "fwd.cuh"
+
+namespace ttt {
+
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 384;    // 12 warps
+constexpr int kGemmEpiWarp0 = 4;
+constexpr int kGemmMaxProblems = 3;
+
+enum GemmEpilogue { kEpiStore = 0, kEpiResidual = 1, kEpiL2Heads = 2, kEpiGate = 3, kEpiDz = 4, kEpiAccF32 = 5 };
+
+struct GemmProblem {
+  int M, N;          // output extent
+  int K;             // reduction length (the maps' extent along K; TMA zero-fills past it)
+  int splits;        // K splits (kEpiAccF32 only; otherwise 1)
+  int k_per_split;   // multiple of kGemmBK
+  int a_mn, b_mn;    // operand layouts: 1 = MN-major
+  int a_x0, a_y0;    // coordinate offsets of the A map (x = inner dimension)
+  int b_x0, b_y0;    // likewise B
+  // epilogue operands
+  void* out;         // bf16, or f32 for kEpiAccF32
+  long long ldo;     // row pitch of out in elements
+  int out_col0;      // column offset inside out's rows
+  const __nv_bfloat16* res;   // kEpiResidual: [rows][ldr] at column res_col0
+  long long ldr;
+  int res_col0;
+  __nv_bfloat16* f1;          // kEpiGate: F1 out (may be null); kEpiDz: F1 in / dZ1 out
+  __nv_bfloat16* f3;          // likewise F3 / dZ3
+  long long ldf;              // row pitch of A, F1, F3 (hidden units)
+  int norm_cols;              // kEpiL2Heads: columns [0, norm_cols) are normalised per 64
+  int accumulate;             // kEpiAccF32: add to out instead of overwriting
+  long long split_stride;     // kEpiAccF32: elements between the partials of consecutive splits
+  int tiles_m, tiles_n;       // filled by the host
+  long long items;            // tiles_m * tiles_n * splits
+};
+
+struct GemmParams {
+  GemmProblem prob[kGemmMaxProblems];
+  int n_problems;
+  long long total_items;
+  unsigned int* status;
+  long long wait_clocks;      // limit of a bounded wait (<= 0: the default)
+};
+
+struct GemmLayout {
+  static constexpr uint32_t kA = kGemmBM * kGemmBK * 2;   // 16 KiB
+  static constexpr uint32_t kB = kGemmBN * kGemmBK * 2;   // 32 KiB
+  static constexpr uint32_t kStage = kA + kB;
+  static constexpr uint32_t off_bar = kGemmStages * kStage;
+  static constexpr int kNumBars = 2 * kGemmStages + 4 + 1;
+  static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
+};
+
+// Work item -> (problem, tile m, tile n, split); tiles of one M row are
+// consecutive, so the CTAs that run at the same time share their A rows in L2.
+struct GemmItem {
+  int p, tm, tn, s;
+};
+__device__ __forceinline__ GemmItem gemm_item(const GemmParams& P, long long it) {
+  GemmItem w{0, 0, 0, 0};
+  int p = 0;
+  while (p + 1 < P.n_problems && it >= P.prob[p].items) {
+    it -= P.prob[p].items;
+    ++p;
+  }
+  const GemmProblem& q = P.prob[p];
+  w.p = p;
+  const long long per_s = static_cast<long long>(q.tiles_m) * q.tiles_n;
+  w.s = static_cast<int>(it / per_s);
+  const long long r = it % per_s;
+  w.tm = static_cast<int>(r / q.tiles_n);
+  w.tn = static_cast<int>(r % q.tiles_n);
+  return w;
+}
+
+__device__ __forceinline__ void gemm_k_range(const GemmProblem& q, int s, int* k0, int* nkb) {
+  const int lo = s * q.k_per_split;
+  int hi = lo + q.k_per_split;
+  if (hi > q.K) hi = q.K;
+  *k0 = lo;
+  *nkb = hi > lo ? (hi - lo + kGemmBK - 1) / kGemmBK : 0;
+}
+
+__device__ __forceinline__ uint32_t gemm_idesc(int a_mn, int b_mn) {
+  return idesc_bf16(kGemmBM, kGemmBN, a_mn != 0, b_mn != 0);
+}
+
+// 32 lanes x 32 bits, 32 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ float gemm_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x);
+  v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z);
+  v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tma0, const __grid_constant__ CUtensorMap tmb0,
+                const __grid_constant__ CUtensorMap tma1, const __grid_constant__ CUtensorMap tmb1,
+                const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2,
+                const __grid_constant__ GemmParams P) {
+  using L = GemmLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kGemmStages;
+  uint64_t* acc_full = bars + 2 * kGemmStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const Abort ab{abort_flag, P.status, P.wait_clocks};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const CUtensorMap* ma[3] = {&tma0, &tma1, &tma2};
+      const CUtensorMap* mb[3] = {&tmb0, &tmb1, &tmb2};
+      for (int p = 0; p < P.n_problems; ++p) {
+        tma_prefetch_desc(ma[p]);
+        tma_prefetch_desc(mb[p]);
+      }
+      uint32_t stage = 0, ph = 0, issued = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < P.total_items && ok; it += gridDim.x) {
+        const GemmItem w = gemm_item(P, it);
+        const GemmProblem& q = P.prob[w.p];
+        int k0, nkb;
+        gemm_k_range(q, w.s, &k0, &nkb);
+        const int m0 = w.tm * kGemmBM, n0 = w.tn * kGemmBN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int k = k0 + kb * kGemmBK;
+          if (!(ok = mbar_wait(&empty[stage], ph ^ 1, ab))) break;
+          mbar_arrive_expect_tx(&full[stage], L::kStage);
+          uint8_t* sa = smem + stage * L::kStage;
+          uint8_t* sb = sa + L::kA;
+          if (q.a_mn) {
+            tma_load_2d(sa, ma[w.p], &full[stage], q.a_x0 + m0, q.a_y0 + k);
+            tma_load_2d(sa + 8192, ma[w.p], &full[stage], q.a_x0 + m0 + 64, q.a_y0 + k);
+          } else {
+            tma_load_2d(sa, ma[w.p], &full[stage], q.a_x0 + k, q.a_y0 + m0);
+          }
+          if (q.b_mn) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tma_load_2d(sb + i * 8192, mb[w.p], &full[stage], q.b_x0 + n0 + 64 * i, q.b_y0 + k);
+          } else {
+            tma_load_2d(sb, mb[w.p], &full[stage], q.b_x0 + k, q.b_y0 + n0);
+            tma_load_2d(sb + 16384, mb[w.p], &full[stage], q.b_x0 + k, q.b_y0 + n0 + 128);
+          }
+          ++issued;
+          if (++stage == kGemmStages) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      // Drain: the last load issued into each stage has landed before exit.
+      const uint32_t last = issued < static_cast<uint32_t>(kGemmStages) ? issued : kGemmStages;
+      for (uint32_t b = 0; b < last; ++b) {
+        const uint32_t jj = issued - 1 - b;
+        mbar_drain(&full[jj % kGemmStages], (jj / kGemmStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t stage = 0, ph = 0, local = 0;
+    bool ok = true;
+    for (long long it = blockIdx.x; it < P.total_items && ok; it += gridDim.x, ++local) {
+      const GemmItem w = gemm_item(P, it);
+      const GemmProblem& q = P.prob[w.p];
+      int k0, nkb;
+      gemm_k_range(q, w.s, &k0, &nkb);
+      const uint32_t buf = local & 1;
+      if (!(ok = mbar_wait_warp(&acc_empty[buf], ((local >> 1) & 1) ^ 1, ab))) break;
+      tc_fence_after();
+      const uint32_t idesc = gemm_idesc(q.a_mn, q.b_mn);
+      // per K=16 step: K-major operands advance 32 bytes, MN-major ones 16 rows of 128 bytes
+      const uint32_t a_step = q.a_mn ? 2048u : 32u, b_step = q.b_mn ? 2048u : 32u;
+      const uint32_t a_lbo = q.a_mn ? 8192u : 16u, b_lbo = q.b_mn ? 8192u : 16u;
+      const uint32_t tacc = tbase + buf * kGemmBN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!(ok = mbar_wait_warp(&full[stage], ph, ab))) break;
+        tc_fence_after();
+        const uint32_t sa = sbase + stage * L::kStage, sb = sa + L::kA;
+        const uint64_t ad = smem_desc(sa, a_lbo, 1024, 128), bd = smem_desc(sb, b_lbo, 1024, 128);
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 16; ++k)
+          mma_bf16_warp(tacc, ad + ((k * a_step) >> 4), bd + ((k * b_step) >> 4), idesc,
+                        (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit_warp(&empty[stage]);
+        if (++stage == kGemmStages) {
+          stage = 0;
+          ph ^= 1;
+        }
+      }
+      if (ok) mma_commit_warp(&acc_full[buf]);
+    }
+    // All issued MMAs have completed before TMEM is released.
+    mma_commit_warp(done);
+    mbar_drain(done, 0);
+  } else if (warp >= kGemmEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - kGemmEpiWarp0;      // 0..7
+    const int quad = warp & 3;               // TMEM lane quadrant
+    const int hf = e >> 2;                   // column half of the tile
+    const int row = quad * 32 + lane;        // row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    uint32_t local = 0;
+    for (long long it = blockIdx.x; it < P.total_items; it += gridDim.x, ++local) {
+      const GemmItem w = gemm_item(P, it);
+      const GemmProblem& q = P.prob[w.p];
+      const uint32_t buf = local & 1;
+      if (!mbar_wait_warp(&acc_full[buf], (local >> 1) & 1, ab)) break;
+      tc_fence_after();
+      const uint32_t tacc = tbase + buf * kGemmBN + lane_off;
+      const long long m = static_cast<long long>(w.tm) * kGemmBM + row;
+      const bool row_ok = m < q.M;
+      const int n0 = w.tn * kGemmBN;
+      if (EPI == kEpiGate) {
+        // hidden units [64 hf, 64 hf + 64) of this tile: Z1 at columns c, Z3 at 128 + c
+        const int hid0 = w.tn * 128 + hf * 64;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          uint32_t z1[32], z3[32];
+          tmem_ld32(tacc + hf * 64 + c0, z1);
+          tmem_ld32(tacc + 128 + hf * 64 + c0, z3);
+          tmem_wait_ld();
+          const int hid = hid0 + c0;
+          if (row_ok && hid < q.N / 2) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float a[8], f1[8], f3[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float x1 = __uint_as_float(z1[8 * g + i]), x3 = __uint_as_float(z3[8 * g + i]);
+                const float s = gemm_sigmoid(x1);
+                const float silu = x1 * s;
+                a[i] = silu * x3;
+                f3[i] = silu;
+                f1[i] = x3 * s * (1.f + x1 * (1.f - s));
+              }
+              const long long off = m * q.ldf + hid + 8 * g;
+              store_bf16x8(reinterpret_cast<__nv_bfloat16*>(q.out) + off, a);
+              if (q.f1) store_bf16x8(q.f1 + off, f1);
+              if (q.f3) store_bf16x8(q.f3 + off, f3);
+            }
+          }
+        }
+      } else if (EPI == kEpiAccF32) {
+        float* out = reinterpret_cast<float*>(q.out) + static_cast<long long>(w.s) * q.split_stride;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tacc + hf * 128 + c0, r);
+          tmem_wait_ld();
+          const int col = n0 + hf * 128 + c0;
+          if (row_ok && col < q.N) {
+            float4* dst = reinterpret_cast<float4*>(out + m * q.ldo + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (col + 4 * v >= q.N) break;   // N is a multiple of 4
+              float4 x = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+              if (q.accumulate) {
+                const float4 o = dst[v];
+                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+              }
+              dst[v] = x;
+            }
+          }
+        }
+      } else if (EPI == kEpiL2Heads) {
+        // two heads of 64 columns per half
+#pragma unroll 1
+        for (int hd = 0; hd < 2; ++hd) {
+          uint32_t r0[32], r1[32];
+          const int c = hf * 128 + hd * 64;
+          tmem_ld32(tacc + c, r0);
+          tmem_ld32(tacc + c + 32, r1);
+          tmem_wait_ld();
+          const int col = n0 + c;
+          if (row_ok && col < q.N) {
+            float scale = 1.f;
+            if (col < q.norm_cols) {
+              float ss = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float a = __uint_as_float(r0[i]), b = __uint_as_float(r1[i]);
+                ss = fmaf(a, a, ss);
+                ss = fmaf(b, b, ss);
+              }
+              scale = ss > 0.f ? rsqrtf(ss) : 0.f;
+            }
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(q.out) + m * q.ldo + q.out_col0 + col;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[8 * g + i]) * scale;
+              store_bf16x8(dst + 8 * g, v);
+            }
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r1[8 * g + i]) * scale;
+              store_bf16x8(dst + 32 + 8 * g, v);
+            }
+          }
+        }
+      } else {
+        // kEpiStore, kEpiResidual, kEpiDz: 128 columns of this half in chunks of 32
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tacc + hf * 128 + c0, r);
+          tmem_wait_ld();
+          const int col = n0 + hf * 128 + c0;
+          if (row_ok && col < q.N) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (col + 8 * g >= q.N) break;   // N is a multiple of 8
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[8 * g + i]);
+              if (EPI == kEpiDz) {
+                const long long off = m * q.ldf + col + 8 * g;
+                float f1[8], f3[8], d1[8], d3[8];
+                load_bf16x8(q.f1 + off, f1);
+                load_bf16x8(q.f3 + off, f3);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  d1[i] = v[i] * f1[i];
+                  d3[i] = v[i] * f3[i];
+                }
+                store_bf16x8(q.f1 + off, d1);
+                store_bf16x8(q.f3 + off, d3);
+              } else {
+                if (EPI == kEpiResidual) {
+                  float rr[8];
+                  load_bf16x8(q.res + m * q.ldr + q.res_col0 + col + 8 * g, rr);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) v[i] -= rr[i];
+                }
+                store_bf16x8(reinterpret_cast<__nv_bfloat16*>(q.out) + m * q.ldo + q.out_col0 + col + 8 * g, v);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace ttt

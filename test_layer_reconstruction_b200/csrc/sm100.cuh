@@ -15,7 +15,8 @@ enum : uint32_t {
   kStatusWaitTimeout = 1u,   // a bounded mbarrier wait ran out
 };
 
-// A bounded wait gives up after this many SM clocks (~2-4 s at B200 clocks).
+// A bounded wait gives up after this many SM clocks (~2-4 s at B200 clocks)
+// unless the launch asks for another limit (Abort::limit).
 constexpr long long kWaitClockLimit = 4000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -70,6 +71,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 struct Abort {
   volatile int* flag;       // shared memory
   unsigned int* status;     // global (may be null)
+  long long limit;          // SM clocks a wait may take; <= 0 means kWaitClockLimit
   __device__ __forceinline__ bool raised() const { return *flag != 0; }
   __device__ __forceinline__ void raise(uint32_t bits) const {
     *flag = 1;
@@ -78,15 +80,16 @@ struct Abort {
 };
 
 // Wait until the phase of `bar` with the given parity has completed.
-// Bounded: returns false (and raises abort) after kWaitClockLimit clocks or
-// when another role already aborted.
+// Bounded: returns false (and raises abort) after the launch's limit of
+// clocks or when another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = ab.limit > 0 ? ab.limit : kWaitClockLimit;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (ab.raised()) return false;
-    if (clock64() - t0 > kWaitClockLimit) {
+    if (clock64() - t0 > limit) {
       ab.raise(kStatusWaitTimeout);
       return false;
     }

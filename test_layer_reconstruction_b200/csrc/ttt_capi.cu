@@ -3,13 +3,14 @@
 //   conv -> steps x [pack theta -> forward (residual) -> backward (partials)
 //   -> reduce + SGD] -> pack theta* -> forward (read)
 // for head widths 16, 32, 64 (h <= 256), and the wide-head sequence (token
-// chunks of bf16 library GEMMs and the elementwise kernels of wide.cuh) for
-// head widths and hidden widths that are multiples of 64 beyond that.
-#include <cublas_v2.h>
+// chunks of the tensor-core GEMM of gemm.cuh with fused epilogues, and the
+// small kernels of wide.cuh) for head widths and hidden widths that are
+// multiples of 64 beyond that.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -17,6 +18,7 @@
 
 #include "../../include/ttt.h"
 #include "conv.cuh"
+#include "gemm.cuh"
 #include "update.cuh"
 #include "wide.cuh"
 
@@ -25,18 +27,17 @@ using namespace ttt;
 namespace {
 
 constexpr size_t kAlign = 1024;
-constexpr int kMaxDevicesWide = 64;
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
 struct Shape {
   long long n;   // tokens
   int H, D, h, hidp, tiles, slices, units;
   long long C;   // H * D channels
-  bool wide;     // wide-head path (library GEMMs over token chunks)
+  bool wide;     // wide-head path (tensor-core GEMMs over token chunks)
 };
 
-constexpr long long kWideChunk = 131072;           // tokens per GEMM chunk of the wide path
-constexpr size_t kWideGemmWorkspace = 32u << 20;   // library GEMM workspace (bytes)
+constexpr long long kWideChunk = 262144;   // tokens per GEMM chunk of the wide path
+constexpr int kWideMaxSplits = 8;          // most K splits of the weight-gradient GEMMs
 
 int check_dims(const ttt_dims* dm, Shape* s) {
   if (!dm) return TTT_EINVAL;
@@ -96,7 +97,7 @@ Grids grids_for(const Shape& s, int sms) {
 
 struct Ws {
   size_t status, w13, w2h, wt, vp, e, part, grad, q, k, v, o, convw, th0, thout, total;
-  size_t img, acc, z1, z3, da, ab, eb, gemm;   // wide path
+  size_t img, img2, acc, z1, z3, ab, eb;   // wide path
 };
 
 Ws ws_layout(const Shape& s, const Grids& g, int op) {
@@ -114,15 +115,14 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
   if (s.wide) {
     const bool writes = op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST;
     const size_t nc = static_cast<size_t>(std::min<long long>(s.n, kWideChunk));
-    w.img = take(3ull * s.H * s.D * s.h * 2);
-    w.z1 = take(nc * s.h * 2);
-    w.z3 = take(nc * s.h * 2);
-    w.ab = take(nc * s.h * 2);
-    w.gemm = take(kWideGemmWorkspace);
+    w.img = take(static_cast<size_t>(s.H) * s.D * 2 * s.hidp * 2);   // per head [d][2 hidp]: W1 | W3 by 128
+    w.img2 = take(static_cast<size_t>(s.H) * s.h * s.D * 2);         // per head [h][d]: W2
+    w.ab = take(nc * s.hidp * 2);                                     // A = silu(Z1) Z3
     if (writes) {
-      w.acc = take(3ull * s.D * s.h * 4);
-      w.da = take(nc * s.h * 2);
-      w.eb = take(nc * s.D * 2);
+      w.z1 = take(nc * s.hidp * 2);                                   // F1, then dZ1
+      w.z3 = take(nc * s.hidp * 2);                                   // F3, then dZ3
+      w.eb = take(nc * s.D * 2);                                      // E = Y - V'
+      w.acc = take(static_cast<size_t>(kWideMaxSplits) * 3 * s.D * s.h * 4);
       w.vp = take(tok_bytes);
     }
     if (op == TTT_OP_LAYER_HOST) {
@@ -139,7 +139,7 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
   }
   w.w13 = take(static_cast<size_t>(s.H) * 2 * s.hidp * s.D * 2);
   w.w2h = take(static_cast<size_t>(s.H) * s.hidp * s.D * 2);
-  if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST) {
+  if (op == TTT_OP_WRITE || op == TTT_OP_LAYER || op == TTT_OP_LAYER_HOST || op == TTT_OP_ATTENTION) {
     w.wt = take(static_cast<size_t>(s.H) * s.hidp * 3 * s.D * 2);
     w.vp = take(tok_bytes);
     w.e = take(tok_bytes);
@@ -154,6 +154,12 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
     w.convw = take(static_cast<size_t>(s.C) * 9 * 4);
     w.th0 = take(theta_bytes);
     w.thout = take(theta_bytes);
+  }
+  if (op == TTT_OP_ATTENTION) {   // q, k, v of the projection and the layer's read O
+    w.q = take(tok_bytes);
+    w.k = take(tok_bytes);
+    w.v = take(tok_bytes);
+    w.o = take(tok_bytes);
   }
   w.total = off;
   return w;
@@ -193,9 +199,13 @@ bool make_token_map(CUtensorMap* m, const void* base, const Shape& s, int rows =
 }
 
 // ------------------------------------------------------------------ profiling
-enum KernelKind { KK_CONV = 0, KK_PACK = 1, KK_FWD_WRITE = 2, KK_BWD = 3, KK_REDUCE = 4, KK_FWD_READ = 5 };
-const char* const kKernelNames[TTT_KERNEL_KINDS] = {"shortconv2d", "pack_theta", "swiglu_fwd_residual",
-                                                     "swiglu_bwd_partials", "reduce_sgd", "swiglu_fwd_read"};
+enum KernelKind {
+  KK_CONV = 0, KK_PACK = 1, KK_FWD_WRITE = 2, KK_BWD = 3, KK_REDUCE = 4, KK_FWD_READ = 5,
+  KK_GEMM_GATE = 6, KK_GEMM_RESIDUAL = 7, KK_GEMM_DZ = 8, KK_GEMM_WGRAD = 9, KK_GEMM_STORE = 10, KK_GEMM_QKV = 11
+};
+const char* const kKernelNames[TTT_KERNEL_KINDS] = {
+    "shortconv2d", "pack_theta", "swiglu_fwd_residual", "swiglu_bwd_partials", "reduce_sgd", "swiglu_fwd_read",
+    "gemm_gate", "gemm_residual", "gemm_dz", "gemm_wgrad", "gemm_store", "gemm_qkv_l2norm"};
 constexpr size_t kMaxProfiled = 65536;
 
 struct Profiler {
@@ -238,6 +248,14 @@ struct ProfScope {
     if (end) cudaEventRecord(end, st);
   }
 };
+
+// Limit (SM clocks) of every bounded wait in the kernels launched from now
+// on; 0 selects the built-in limit.  Set by ttt_set_wait_limit.
+std::atomic<long long>& wait_clock_setting() {
+  static std::atomic<long long> v{0};
+  return v;
+}
+long long wait_clocks() { return wait_clock_setting().load(std::memory_order_relaxed); }
 
 bool aligned(const void* p, size_t a = 16) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -361,119 +379,231 @@ int prepare(const ttt_dims* dm, int op, void* workspace, size_t ws_bytes, void* 
   return TTT_OK;
 }
 
-// ------------------------------------------------------------------ wide path
-// One library GEMM handle per device, created on first use; enqueues of the
-// wide path on a device are serialised because the handle's stream and
-// workspace are set per call.
-struct WideGemm {
-  std::mutex mu;
-  cublasHandle_t h[kMaxDevicesWide] = {};
-};
-WideGemm& wide_gemm() {
-  static WideGemm g;
-  return g;
+// ------------------------------------------------------------------ tensor-core GEMM
+// 2-D bf16 tensor [rows][cols] (row pitch `pitch` elements) for the GEMM's
+// operand loads: K-major boxes are 64 columns x 128 rows, MN-major boxes 64
+// columns x 64 rows, both with the 128-byte swizzle.
+bool make_gemm_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, bool mn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows < 1 || cols < 1) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch) * 2};
+  cuuint32_t box[2] = {64u, mn ? 64u : 128u};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major C[M x N] (ldc) = alpha op(A)[M x K] op(B)[K x N] + beta C, bf16 A and
-// B, FP32 accumulation; op(A) = A^T when `ta` (A stored K x M), likewise B.
-// Column-major view: C^T = op(B)^T op(A)^T.
-bool gemm_rm(cublasHandle_t hd, bool ta, bool tb, int M, int N, int K, float alpha, const void* A, int lda,
-             const void* B, int ldb, float beta, void* C, cudaDataType_t ctype, int ldc) {
-  return cublasGemmEx(hd, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, B,
-                      CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda, &beta, C, ctype, ldc, CUBLAS_COMPUTE_32F,
-                      CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
-}
-
-unsigned elementwise_grid(long long n8) {
-  const int sms = num_sms();
-  return static_cast<unsigned>(std::max<long long>(1, std::min<long long>((n8 + 255) / 256, 8LL * (sms > 0 ? sms : 148))));
-}
-
-// Takes the device's GEMM handle (created on first use) bound to this call's
-// stream and workspace; holds the device's lock for the caller's enqueue.
-struct WideCall {
-  std::unique_lock<std::mutex> lock;
-  cublasHandle_t hd = nullptr;
-  bool ok = false;
-  WideCall(const Call& c) : lock(wide_gemm().mu) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesWide) return;
-    cublasHandle_t& h = wide_gemm().h[dev];
-    if (!h && cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) {
-      h = nullptr;
-      return;
-    }
-    if (cublasSetStream(h, c.st) != CUBLAS_STATUS_SUCCESS) return;
-    if (cublasSetWorkspace(h, c.ws + c.w.gemm, kWideGemmWorkspace) != CUBLAS_STATUS_SUCCESS) return;
-    hd = h;
-    ok = true;
+// One launch of gemm_kernel: up to three problems with their operand maps.
+struct GemmLaunch {
+  GemmParams P;
+  CUtensorMap ma[kGemmMaxProblems], mb[kGemmMaxProblems];
+  GemmLaunch() {
+    memset(&P, 0, sizeof(P));
+    memset(ma, 0, sizeof(ma));
+    memset(mb, 0, sizeof(mb));
+  }
+  // A problem of M x N with reduction length K; `splits` > 1 only for kEpiAccF32.
+  GemmProblem& add(int M, int N, int K, bool a_mn, bool b_mn, int splits = 1) {
+    GemmProblem& q = P.prob[P.n_problems++];
+    q.M = M;
+    q.N = N;
+    q.K = K;
+    q.a_mn = a_mn;
+    q.b_mn = b_mn;
+    const int kblocks = (K + kGemmBK - 1) / kGemmBK;
+    splits = std::max(1, std::min(splits, kblocks));
+    q.k_per_split = (kblocks + splits - 1) / splits * kGemmBK;
+    q.splits = (K + q.k_per_split - 1) / q.k_per_split;
+    q.tiles_m = (M + kGemmBM - 1) / kGemmBM;
+    q.tiles_n = (N + kGemmBN - 1) / kGemmBN;
+    q.items = static_cast<long long>(q.tiles_m) * q.tiles_n * q.splits;
+    return q;
   }
 };
 
-int wide_cast(const Call& c, const float* theta) {
-  const long long count = 3LL * c.s.H * c.s.D * c.s.h;
-  wide_cast_kernel<<<elementwise_grid(count / 8), 256, 0, c.st>>>(
-      theta, reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.img), count);
+template <int EPI>
+int launch_gemm(GemmLaunch& g, unsigned int* status, int kind, cudaStream_t st) {
+  g.P.status = status;
+  g.P.wait_clocks = wait_clocks();
+  g.P.total_items = 0;
+  for (int p = 0; p < g.P.n_problems; ++p) g.P.total_items += g.P.prob[p].items;
+  if (g.P.total_items == 0) return TTT_OK;
+  for (int p = g.P.n_problems; p < kGemmMaxProblems; ++p) {
+    g.ma[p] = g.ma[0];
+    g.mb[p] = g.mb[0];
+  }
+  const int sms = num_sms();
+  const int grid = static_cast<int>(std::min<long long>(sms > 0 ? sms : 148, g.P.total_items));
+  auto k = gemm_kernel<EPI>;
+  const uint32_t smem = GemmLayout::bytes;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return TTT_ECUDA;
+  ProfScope prof(kind, st);
+  k<<<grid, kGemmThreads, smem, st>>>(g.ma[0], g.mb[0], g.ma[1], g.mb[1], g.ma[2], g.mb[2], g.P);
   return launch_status();
 }
 
-// Z1, Z3 (bf16) of rows [t0, t0 + nc) of head hd of X, then A = silu(Z1) Z3.
-int wide_forward_chunk(const Call& c, cublasHandle_t hd, const uint16_t* X, int head, long long t0, int nc) {
+// K splits of the weight-gradient launch: enough items for about three waves
+// of one CTA per SM.
+int wgrad_splits(const Shape& s, long long nc) {
+  const int sms = std::max(1, num_sms());
+  const long long tiles = 2LL * ((s.D + kGemmBM - 1) / kGemmBM) * ((s.h + kGemmBN - 1) / kGemmBN) +
+                          static_cast<long long>((s.h + kGemmBM - 1) / kGemmBM) * ((s.D + kGemmBN - 1) / kGemmBN);
+  const long long want = (3LL * sms + tiles - 1) / tiles;
+  const long long kblocks = (nc + kGemmBK - 1) / kGemmBK;
+  return static_cast<int>(std::max<long long>(1, std::min<long long>({want, kWideMaxSplits, kblocks})));
+}
+
+// ------------------------------------------------------------------ the layer's surround
+// q = L2(X Wq), k = L2(X Wk) per (token, head) row of 64, v = X Wv: one launch
+// of three problems sharing the A operand X.
+int run_qkv(const Call& c, const uint16_t* X, const uint16_t* Wq, const uint16_t* Wk, const uint16_t* Wv,
+            uint16_t* q, uint16_t* k, uint16_t* v) {
   const Shape& s = c.s;
-  const size_t per = static_cast<size_t>(s.D) * s.h;
-  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
-  const uint16_t* xc = X + (static_cast<size_t>(t0) * s.H + head) * s.D;
-  const int ldx = s.H * s.D;
-  if (!gemm_rm(hd, false, false, nc, s.h, s.D, 1.f, xc, ldx, img + head * per, s.h, 0.f, c.ws + c.w.z1, CUDA_R_16BF,
-               s.h) ||
-      !gemm_rm(hd, false, false, nc, s.h, s.D, 1.f, xc, ldx, img + (s.H + head) * per, s.h, 0.f, c.ws + c.w.z3,
-               CUDA_R_16BF, s.h))
+  GemmLaunch g;
+  const uint16_t* W[3] = {Wq, Wk, Wv};
+  uint16_t* out[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    if (!make_gemm_map(&g.ma[i], X, s.n, s.C, s.C, false) || !make_gemm_map(&g.mb[i], W[i], s.C, s.C, s.C, true))
+      return TTT_ECUDA;
+    GemmProblem& p = g.add(static_cast<int>(s.n), static_cast<int>(s.C), static_cast<int>(s.C), false, true);
+    p.out = out[i];
+    p.ldo = s.C;
+    p.norm_cols = i < 2 ? static_cast<int>(s.C) : 0;
+  }
+  return launch_gemm<kEpiL2Heads>(g, reinterpret_cast<unsigned int*>(c.ws + c.w.status), KK_GEMM_QKV, c.st);
+}
+
+// out = O Wo.
+int run_out_proj(const Call& c, const uint16_t* O, const uint16_t* Wo, uint16_t* out) {
+  const Shape& s = c.s;
+  GemmLaunch g;
+  if (!make_gemm_map(&g.ma[0], O, s.n, s.C, s.C, false) || !make_gemm_map(&g.mb[0], Wo, s.C, s.C, s.C, true))
     return TTT_ECUDA;
-  const long long n8 = static_cast<long long>(nc) * s.h / 8;
-  wide_gate_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<const uint4*>(c.ws + c.w.z1),
-                                                           reinterpret_cast<const uint4*>(c.ws + c.w.z3),
-                                                           reinterpret_cast<uint4*>(c.ws + c.w.ab), n8);
+  GemmProblem& p = g.add(static_cast<int>(s.n), static_cast<int>(s.C), static_cast<int>(s.C), false, true);
+  p.out = out;
+  p.ldo = s.C;
+  return launch_gemm<kEpiStore>(g, reinterpret_cast<unsigned int*>(c.ws + c.w.status), KK_GEMM_STORE, c.st);
+}
+
+// ------------------------------------------------------------------ wide path
+unsigned elementwise_grid(long long n) {
+  const int sms = num_sms();
+  return static_cast<unsigned>(std::max<long long>(1, std::min<long long>((n + 255) / 256, 8LL * (sms > 0 ? sms : 148))));
+}
+
+// Operand images of theta for the wide path: per head W13 [d][2 hidp] (hidden
+// block j of 128 units: W1 columns, then W3 columns) and W2 [h][d], bf16.
+int wide_pack(const Call& c, const float* theta) {
+  const Shape& s = c.s;
+  const long long count = static_cast<long long>(s.H) * s.D * (2LL * s.hidp + s.h);
+  ProfScope prof(KK_PACK, c.st);
+  wide_pack_kernel<<<elementwise_grid(count), 256, 0, c.st>>>(
+      theta, reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.img), reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.img2),
+      s.H, s.D, s.h, s.hidp);
   return launch_status();
 }
 
-// dW of one head of the wide path over all tokens, per token chunk
-//   Z1, Z3, A (forward) -> E = A W2 - V' -> dA = E W2^T -> dZ1, dZ3
-//   -> dW1 += K^T dZ1, dW3 += K^T dZ3, dW2 += A^T E   (FP32, Eq. 5)
-// into the workspace accumulator; the operand image of theta is current.
-int wide_grad_head(const Call& c, cublasHandle_t hd, const uint16_t* K, const uint16_t* vp, int head) {
+struct WideOperands {
+  const __nv_bfloat16* img13;   // this head's W13 image
+  const __nv_bfloat16* img2;    // this head's W2 image
+};
+WideOperands wide_head(const Call& c, int head) {
   const Shape& s = c.s;
-  const size_t per = static_cast<size_t>(s.D) * s.h;
-  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
+  WideOperands o;
+  o.img13 = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img) + static_cast<size_t>(head) * s.D * 2 * s.hidp;
+  o.img2 = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img2) + static_cast<size_t>(head) * s.h * s.D;
+  return o;
+}
+
+// Gate of rows [t0, t0 + nc) of head `head` of X: A = silu(X W1) (X W3), and
+// with `chain` also F1, F3 (the backward's chain-rule factors).
+int wide_gate_chunk(const Call& c, const uint16_t* X, int head, long long t0, int nc, bool chain) {
+  const Shape& s = c.s;
+  const WideOperands w = wide_head(c, head);
+  GemmLaunch g;
+  if (!make_gemm_map(&g.ma[0], X + static_cast<size_t>(t0) * s.C, nc, s.C, s.C, false) ||
+      !make_gemm_map(&g.mb[0], w.img13, s.D, 2LL * s.hidp, 2LL * s.hidp, true))
+    return TTT_ECUDA;
+  GemmProblem& q = g.add(nc, 2 * s.hidp, s.D, false, true);
+  q.a_x0 = head * s.D;
+  q.out = c.ws + c.w.ab;
+  q.ldf = s.hidp;
+  q.f1 = chain ? reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.z1) : nullptr;
+  q.f3 = chain ? reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.z3) : nullptr;
+  return launch_gemm<kEpiGate>(g, reinterpret_cast<unsigned int*>(c.ws + c.w.status), KK_GEMM_GATE, c.st);
+}
+
+// dW of one head of the wide path over all tokens, per token chunk:
+//   A, F1, F3 (gate GEMM) -> E = A W2 - V' -> dA = E W2^T, dZ1 = dA F1, dZ3 = dA F3
+//   -> dW1 += K^T dZ1, dW3 += K^T dZ3, dW2 += A^T E   (FP32 split-K partials, Eq. 5)
+// into the workspace accumulator [splits][dW1 | dW3 | dW2]; returns the split count.
+int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int head, int* splits_out) {
+  const Shape& s = c.s;
+  const WideOperands w = wide_head(c, head);
+  unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
   float* acc = reinterpret_cast<float*>(c.ws + c.w.acc);
-  uint8_t* eb = c.ws + c.w.eb;
-  const int ldx = s.H * s.D;
-  const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;   // [h][D]
-  int rc;
+  __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.ab);
+  __nv_bfloat16* f1 = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.z1);
+  __nv_bfloat16* f3 = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.z3);
+  __nv_bfloat16* eb = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.eb);
+  const long long per = static_cast<long long>(s.D) * s.h;
+  int rc, splits = 1;
   for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
     const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
-    const float beta = t0 == 0 ? 0.f : 1.f;
-    if ((rc = wide_forward_chunk(c, hd, K, head, t0, nc)) != TTT_OK) return rc;
-    // E = A W2 - V' (the chunk's V' rows first copied into E)
-    if (cudaMemcpy2DAsync(eb, static_cast<size_t>(s.D) * 2, vp + (static_cast<size_t>(t0) * s.H + head) * s.D,
-                          static_cast<size_t>(ldx) * 2, static_cast<size_t>(s.D) * 2, nc, cudaMemcpyDeviceToDevice,
-                          c.st) != cudaSuccess)
-      return TTT_ECUDA;
-    if (!gemm_rm(hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, -1.f, eb, CUDA_R_16BF, s.D) ||
-        !gemm_rm(hd, false, true, nc, s.h, s.D, 1.f, eb, s.D, w2, s.D, 0.f, c.ws + c.w.da, CUDA_R_16BF, s.h))
-      return TTT_ECUDA;
-    const long long n8 = static_cast<long long>(nc) * s.h / 8;
-    wide_dz_kernel<<<elementwise_grid(n8), 256, 0, c.st>>>(reinterpret_cast<uint4*>(c.ws + c.w.z1),
-                                                           reinterpret_cast<uint4*>(c.ws + c.w.z3),
-                                                           reinterpret_cast<const uint4*>(c.ws + c.w.da), n8);
-    if ((rc = launch_status()) != TTT_OK) return rc;
-    const uint16_t* kc = K + (static_cast<size_t>(t0) * s.H + head) * s.D;
-    if (!gemm_rm(hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z1, s.h, beta, acc, CUDA_R_32F, s.h) ||
-        !gemm_rm(hd, true, false, s.D, s.h, nc, 1.f, kc, ldx, c.ws + c.w.z3, s.h, beta, acc + per, CUDA_R_32F,
-                 s.h) ||
-        !gemm_rm(hd, true, false, s.h, s.D, nc, 1.f, c.ws + c.w.ab, s.h, eb, s.D, beta, acc + 2 * per, CUDA_R_32F,
-                 s.D))
-      return TTT_ECUDA;
+    if ((rc = wide_gate_chunk(c, K, head, t0, nc, true)) != TTT_OK) return rc;
+    {  // E = A W2 - V'
+      GemmLaunch g;
+      if (!make_gemm_map(&g.ma[0], ab, nc, s.hidp, s.hidp, false) ||
+          !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, true))
+        return TTT_ECUDA;
+      GemmProblem& q = g.add(nc, s.D, s.h, false, true);
+      q.out = eb;
+      q.ldo = s.D;
+      q.res = reinterpret_cast<const __nv_bfloat16*>(vp) + static_cast<size_t>(t0) * s.C;
+      q.ldr = s.C;
+      q.res_col0 = head * s.D;
+      if ((rc = launch_gemm<kEpiResidual>(g, status, KK_GEMM_RESIDUAL, c.st)) != TTT_OK) return rc;
+    }
+    {  // dA = E W2^T, then dZ1 = dA F1, dZ3 = dA F3 in place
+      GemmLaunch g;
+      if (!make_gemm_map(&g.ma[0], eb, nc, s.D, s.D, false) || !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, false))
+        return TTT_ECUDA;
+      GemmProblem& q = g.add(nc, s.hidp, s.D, false, false);
+      q.f1 = f1;
+      q.f3 = f3;
+      q.ldf = s.hidp;
+      if ((rc = launch_gemm<kEpiDz>(g, status, KK_GEMM_DZ, c.st)) != TTT_OK) return rc;
+    }
+    {  // dW1 = K^T dZ1, dW3 = K^T dZ3, dW2 = A^T E, split over the chunk's tokens
+      GemmLaunch g;
+      const uint16_t* kc = K + static_cast<size_t>(t0) * s.C;
+      if (!make_gemm_map(&g.ma[0], kc, nc, s.C, s.C, true) || !make_gemm_map(&g.mb[0], f1, nc, s.hidp, s.hidp, true) ||
+          !make_gemm_map(&g.ma[1], kc, nc, s.C, s.C, true) || !make_gemm_map(&g.mb[1], f3, nc, s.hidp, s.hidp, true) ||
+          !make_gemm_map(&g.ma[2], ab, nc, s.hidp, s.hidp, true) || !make_gemm_map(&g.mb[2], eb, nc, s.D, s.D, true))
+        return TTT_ECUDA;
+      // The first chunk is the largest and fixes the split count: every later
+      // chunk adds its split s into partial s (it may have fewer splits,
+      // whose partials then gain nothing), and the update sums the first
+      // chunk's splits in order.
+      const int sp = t0 == 0 ? wgrad_splits(s, nc) : splits;
+      const int acc_flag = t0 > 0 ? 1 : 0;
+      GemmProblem* qs[3] = {&g.add(s.D, s.h, nc, true, true, sp), &g.add(s.D, s.h, nc, true, true, sp),
+                            &g.add(s.h, s.D, nc, true, true, sp)};
+      if (t0 == 0) splits = qs[0]->splits;
+      for (int m = 0; m < 3; ++m) {
+        GemmProblem& q = *qs[m];
+        q.a_x0 = m < 2 ? head * s.D : 0;
+        q.out = acc + m * per;
+        q.ldo = m < 2 ? s.h : s.D;
+        q.split_stride = 3 * per;
+        q.accumulate = acc_flag;
+      }
+      if ((rc = launch_gemm<kEpiAccF32>(g, status, KK_GEMM_WGRAD, c.st)) != TTT_OK) return rc;
+    }
   }
+  *splits_out = splits;
   return TTT_OK;
 }
 
@@ -491,18 +621,18 @@ int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const u
       return TTT_ECUDA;
     return TTT_OK;
   }
-  WideCall wc(c);
-  if (!wc.ok) return TTT_ECUDA;
-  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const long long per = static_cast<long long>(s.D) * s.h;
   const float* acc = reinterpret_cast<const float*>(c.ws + c.w.acc);
   const float scale = lr * 2.0f / static_cast<float>(s.n);
   for (int step = 0; step < steps; ++step) {
     const float* th_in = step == 0 ? theta0 : theta_out;
-    if ((rc = wide_cast(c, th_in)) != TTT_OK) return rc;
+    if ((rc = wide_pack(c, th_in)) != TTT_OK) return rc;
     for (int head = 0; head < s.H; ++head) {
-      if ((rc = wide_grad_head(c, wc.hd, K, vp, head)) != TTT_OK) return rc;
-      wide_sgd_kernel<<<elementwise_grid(static_cast<long long>(3 * per) / 8), 256, 0, c.st>>>(
-          th_in, theta_out, acc, s.H, s.D, s.h, head, scale);
+      int splits = 1;
+      if ((rc = wide_grad_head(c, K, vp, head, &splits)) != TTT_OK) return rc;
+      ProfScope prof(KK_REDUCE, c.st);
+      wide_sgd_kernel<<<elementwise_grid(3 * per), 256, 0, c.st>>>(th_in, theta_out, acc, splits, s.H, s.D, s.h,
+                                                                    head, scale);
       if ((rc = launch_status()) != TTT_OK) return rc;
     }
   }
@@ -512,40 +642,41 @@ int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const u
 // The gradient (1/2) d/dtheta sum_i ||T(k_i) - v'_i||^2 of the wide path.
 int run_grad_wide(const Call& c, const uint16_t* K, const uint16_t* vp, const float* theta, float* grad) {
   const Shape& s = c.s;
-  WideCall wc(c);
-  if (!wc.ok) return TTT_ECUDA;
-  const size_t per = static_cast<size_t>(s.D) * s.h;
+  const long long per = static_cast<long long>(s.D) * s.h;
   const float* acc = reinterpret_cast<const float*>(c.ws + c.w.acc);
-  int rc = wide_cast(c, theta);
+  int rc = wide_pack(c, theta);
   if (rc != TTT_OK) return rc;
   for (int head = 0; head < s.H; ++head) {
-    if ((rc = wide_grad_head(c, wc.hd, K, vp, head)) != TTT_OK) return rc;
-    wide_grad_kernel<<<elementwise_grid(static_cast<long long>(3 * per) / 8), 256, 0, c.st>>>(grad, acc, s.H, s.D,
-                                                                                              s.h, head);
+    int splits = 1;
+    if ((rc = wide_grad_head(c, K, vp, head, &splits)) != TTT_OK) return rc;
+    ProfScope prof(KK_REDUCE, c.st);
+    wide_grad_kernel<<<elementwise_grid(3 * per), 256, 0, c.st>>>(grad, acc, splits, s.H, s.D, s.h, head);
     if ((rc = launch_status()) != TTT_OK) return rc;
   }
   return TTT_OK;
 }
 
-// The read of the wide path: per head and token chunk, Z1, Z3, A, then
-// O = A W2 written straight into the head's columns of O.
+// The read of the wide path: per head and token chunk, the gate GEMM (A),
+// then O = A W2 written straight into the head's columns of O.
 int run_read_wide(const Call& c, const uint16_t* Q, const float* theta, uint16_t* O) {
   const Shape& s = c.s;
-  WideCall wc(c);
-  if (!wc.ok) return TTT_ECUDA;
-  int rc = wide_cast(c, theta);
+  int rc = wide_pack(c, theta);
   if (rc != TTT_OK) return rc;
-  const size_t per = static_cast<size_t>(s.D) * s.h;
-  const __nv_bfloat16* img = reinterpret_cast<const __nv_bfloat16*>(c.ws + c.w.img);
-  const int ldx = s.H * s.D;
+  unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
   for (int head = 0; head < s.H; ++head) {
-    const __nv_bfloat16* w2 = img + (2 * static_cast<size_t>(s.H) + head) * per;
+    const WideOperands w = wide_head(c, head);
     for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
       const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
-      if ((rc = wide_forward_chunk(c, wc.hd, Q, head, t0, nc)) != TTT_OK) return rc;
-      if (!gemm_rm(wc.hd, false, false, nc, s.D, s.h, 1.f, c.ws + c.w.ab, s.h, w2, s.D, 0.f,
-                   O + (static_cast<size_t>(t0) * s.H + head) * s.D, CUDA_R_16BF, ldx))
+      if ((rc = wide_gate_chunk(c, Q, head, t0, nc, false)) != TTT_OK) return rc;
+      GemmLaunch g;
+      if (!make_gemm_map(&g.ma[0], c.ws + c.w.ab, nc, s.hidp, s.hidp, false) ||
+          !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, true))
         return TTT_ECUDA;
+      GemmProblem& q = g.add(nc, s.D, s.h, false, true);
+      q.out = O + static_cast<size_t>(t0) * s.C;
+      q.ldo = s.C;
+      q.out_col0 = head * s.D;
+      if ((rc = launch_gemm<kEpiStore>(g, status, KK_GEMM_STORE, c.st)) != TTT_OK) return rc;
     }
   }
   return TTT_OK;
@@ -579,6 +710,7 @@ bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradP
   fp.heads = s.H;
   fp.tiles = s.tiles;
   fp.status = status;
+  fp.wait_clocks = wait_clocks();
   BwdParams& bp = gp->bp;
   bp.wt_img = reinterpret_cast<const uint32_t*>(c.ws + c.w.wt);
   bp.partials = reinterpret_cast<float*>(c.ws + c.w.part);
@@ -588,6 +720,7 @@ bool setup_grad_pass(const Call& c, const uint16_t* K, const uint16_t* vp, GradP
   bp.slices = s.slices;
   bp.max_contrib = c.g.max_contrib;
   bp.status = status;
+  bp.wait_clocks = wait_clocks();
   UpdateParams& up = gp->up;
   up.partials = bp.partials;
   up.heads = s.H;
@@ -714,6 +847,7 @@ int launch_read_tokens(const Call& c, const uint16_t* Q, uint16_t* O, long long 
   fp.heads = s.H;
   fp.tiles = s.tiles;
   fp.status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
+  fp.wait_clocks = wait_clocks();
   const int grid = static_cast<int>(std::min<long long>(c.g.fwd, static_cast<long long>(s.H) * s.tiles));
   return launch_fwd<false>(s, tq, tq, fp, grid, c.st);
 }
@@ -835,7 +969,7 @@ int ttt_read_noalloc(const ttt_dims* dims, const uint16_t* Q, const float* theta
 size_t ttt_workspace_bytes(const ttt_dims* dims, int op) {
   Shape s;
   if (check_dims(dims, &s) != TTT_OK) return 0;
-  if (op < TTT_OP_WRITE || op > TTT_OP_LAYER_HOST) return 0;
+  if (op < TTT_OP_WRITE || op > TTT_OP_ATTENTION) return 0;
   const int sms = num_sms();
   if (sms <= 0) return 0;
   return ws_layout(s, grids_for(s, sms), op).total;
@@ -964,6 +1098,50 @@ int ttt_layer(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, const 
   return run_read(c, Q, theta_out, O);
 }
 
+int ttt_attention(const ttt_dims* dims, const uint16_t* X, const uint16_t* Wq, const uint16_t* Wk,
+                  const uint16_t* Wv, const uint16_t* Wo, const float* conv_w, const float* theta0, float lr,
+                  int steps, int inner, float* theta_out, uint16_t* out, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (!X || !Wq || !Wk || !Wv || !Wo || !conv_w || !theta0 || !theta_out || !out || steps < 0) return TTT_EINVAL;
+  if (inner != TTT_INNER_SGD && inner != TTT_INNER_MUON) return TTT_EINVAL;
+  if (!aligned(X) || !aligned(Wq) || !aligned(Wk) || !aligned(Wv) || !aligned(Wo) || !aligned(conv_w) ||
+      !aligned(theta0) || !aligned(theta_out) || !aligned(out))
+    return TTT_EALIGN;
+  int rc = fused_only(dims);
+  if (rc != TTT_OK) return rc;
+  if (dims->d != 64) return TTT_EUNSUPPORTED;   // the normalising epilogue takes heads of 64
+  Call c;
+  rc = prepare(dims, TTT_OP_ATTENTION, workspace, workspace_bytes, stream, &c);
+  if (rc != TTT_OK) return rc;
+  uint16_t* q = reinterpret_cast<uint16_t*>(c.ws + c.w.q);
+  uint16_t* k = reinterpret_cast<uint16_t*>(c.ws + c.w.k);
+  uint16_t* v = reinterpret_cast<uint16_t*>(c.ws + c.w.v);
+  uint16_t* o = reinterpret_cast<uint16_t*>(c.ws + c.w.o);
+  if ((rc = run_qkv(c, X, Wq, Wk, Wv, q, k, v)) != TTT_OK) return rc;
+  rc = inner == TTT_INNER_SGD ? run_write(c, dims, k, v, conv_w, theta0, lr, steps, theta_out)
+                              : run_write_muon(c, dims, k, v, conv_w, theta0, lr, steps, theta_out);
+  if (rc != TTT_OK) return rc;
+  if ((rc = run_read(c, q, theta_out, o)) != TTT_OK) return rc;
+  return run_out_proj(c, o, Wo, out);
+}
+
+int ttt_gemm_bf16(int M, int N, int K, const uint16_t* A, int64_t lda, int a_layout, const uint16_t* B, int64_t ldb,
+                  int b_layout, uint16_t* C, int64_t ldc, void* stream) {
+  if (!A || !B || !C || M < 1 || N < 1 || K < 1) return TTT_EINVAL;
+  if ((a_layout != 0 && a_layout != 1) || (b_layout != 0 && b_layout != 1)) return TTT_EINVAL;
+  if (lda < (a_layout ? M : K) || ldb < (b_layout ? K : N) || ldc < N) return TTT_EINVAL;
+  if (!aligned(A) || !aligned(B) || !aligned(C) || lda % 8 || ldb % 8 || ldc % 8 || N % 8) return TTT_EALIGN;
+  GemmLaunch g;
+  const bool a_mn = a_layout == 1, b_mn = b_layout == 0;
+  if (!make_gemm_map(&g.ma[0], A, a_mn ? K : M, a_mn ? M : K, lda, a_mn) ||
+      !make_gemm_map(&g.mb[0], B, b_mn ? K : N, b_mn ? N : K, ldb, b_mn))
+    return TTT_ECUDA;
+  GemmProblem& p = g.add(M, N, K, a_mn, b_mn);
+  p.out = C;
+  p.ldo = ldc;
+  return launch_gemm<kEpiStore>(g, nullptr, KK_GEMM_STORE, static_cast<cudaStream_t>(stream));
+}
+
 int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t* K_host, const uint16_t* V_host,
                    const float* conv_w_host, const float* theta0_host, float lr, int steps, float* theta_out_host,
                    uint16_t* O_host, void* workspace, size_t workspace_bytes, void* stream) {
@@ -1053,6 +1231,12 @@ int ttt_layer_host(const ttt_dims* dims, const uint16_t* Q_host, const uint16_t*
   }
   if (cudaEventRecord(ev_done, hp.down) != cudaSuccess || cudaStreamWaitEvent(c.st, ev_done, 0) != cudaSuccess)
     return TTT_ECUDA;
+  return TTT_OK;
+}
+
+int ttt_set_wait_limit(long long clocks) {
+  if (clocks < 0) return TTT_EINVAL;
+  wait_clock_setting().store(clocks, std::memory_order_relaxed);
   return TTT_OK;
 }
 

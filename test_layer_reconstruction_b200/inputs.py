@@ -41,7 +41,7 @@ from typing import Dict, Iterable, Optional, Sequence
 import torch
 
 __all__ = [
-    "LayerConfig", "CONFIGS", "make_inputs", "pack_theta", "unpack_theta",
+    "LayerConfig", "CONFIGS", "make_inputs", "make_surround", "pack_theta", "unpack_theta",
     "theta_numel", "bf16_round", "view_token_index",
 ]
 
@@ -49,6 +49,7 @@ _MASK64 = (1 << 64) - 1
 
 # tensor ids of the counter-based seeding
 _TID_K, _TID_Q, _TID_V, _TID_CONV, _TID_W1, _TID_W3, _TID_W2, _TID_X = range(8)
+_TID_TOKENS, _TID_WQ, _TID_WK, _TID_WV, _TID_WO = range(8, 13)
 
 
 def _splitmix64(x: int) -> int:
@@ -218,6 +219,27 @@ def make_inputs(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] =
     out["W1"] = _randn((cfg.heads, cfg.d, cfg.h), seed, _TID_W1, 0, device) * std
     out["W3"] = _randn((cfg.heads, cfg.d, cfg.h), seed, _TID_W3, 0, device) * std
     out["W2"] = _randn((cfg.heads, cfg.h, cfg.d), seed, _TID_W2, 0, device) * std
+    return out
+
+
+def make_surround(cfg: LayerConfig, device="cpu", views: Optional[Sequence[int]] = None) -> Dict[str, torch.Tensor]:
+    """Inputs of the attention layer around the TTT layer: token features
+    X [n, C] ~ N(0, 1) and projections Wq, Wk, Wv, Wo [C, C] ~ N(0, 1/C)
+    (C = heads * d; row-vector form x W), all rounded to bfloat16 and returned
+    as float32; plus the layer's conv_w, W1, W3, W2 as in ``make_inputs``."""
+    if views is None:
+        views = range(cfg.n_views)
+    views = list(views)
+    C = cfg.heads * cfg.d
+    parts = [_randn((cfg.tokens_per_view, C), cfg.seed, _TID_TOKENS, v, device) for v in views]
+    out: Dict[str, torch.Tensor] = {"X": bf16_round(torch.cat(parts, 0))}
+    for name, tid in (("Wq", _TID_WQ), ("Wk", _TID_WK), ("Wv", _TID_WV), ("Wo", _TID_WO)):
+        out[name] = bf16_round(_randn((C, C), cfg.seed, tid, 0, device) * (1.0 / math.sqrt(C)))
+    out["conv_w"] = _randn((C, 3, 3), cfg.seed, _TID_CONV, 0, device) * (1.0 / 3.0)
+    std = math.sqrt(2.0 / (cfg.d + cfg.h))
+    out["W1"] = _randn((cfg.heads, cfg.d, cfg.h), cfg.seed, _TID_W1, 0, device) * std
+    out["W3"] = _randn((cfg.heads, cfg.d, cfg.h), cfg.seed, _TID_W3, 0, device) * std
+    out["W2"] = _randn((cfg.heads, cfg.h, cfg.d), cfg.seed, _TID_W2, 0, device) * std
     return out
 
 

@@ -18,16 +18,18 @@ __all__ = [
     "TTTError", "Dims", "library_path", "load_library", "workspace_bytes", "make_workspace",
     "shortconv2d", "write", "grad", "sgd_update", "read", "layer", "layer_host", "check_status",
     "write_muon", "layer_muon", "grad_dot", "muon_update",
-    "OP_WRITE", "OP_READ", "OP_LAYER", "OP_LAYER_HOST", "EXPORTED_SYMBOLS", "profile_start", "profile_stop",
+    "OP_WRITE", "OP_READ", "OP_LAYER", "OP_LAYER_HOST", "OP_ATTENTION", "INNER_SGD", "INNER_MUON",
+    "attention", "gemm_bf16", "set_wait_limit", "EXPORTED_SYMBOLS", "profile_start", "profile_stop",
 ]
 
-OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST = 0, 1, 2, 3
+OP_WRITE, OP_READ, OP_LAYER, OP_LAYER_HOST, OP_ATTENTION = 0, 1, 2, 3, 4
+INNER_SGD, INNER_MUON = 0, 1
 EXPORTED_SYMBOLS = ("ttt_workspace_bytes", "ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer",
                     "ttt_layer_host", "ttt_check_status", "ttt_status_str", "ttt_profile_start",
                     "ttt_profile_stop", "ttt_kernel_name", "ttt_read_noalloc", "ttt_read_noalloc_status",
                     "ttt_grad", "ttt_sgd_update", "ttt_write_muon", "ttt_layer_muon", "ttt_grad_dot",
-                    "ttt_muon_update")
-KERNEL_KINDS = 6
+                    "ttt_muon_update", "ttt_attention", "ttt_gemm_bf16", "ttt_set_wait_limit")
+KERNEL_KINDS = 12
 
 
 class KernelTimes(ctypes.Structure):
@@ -91,6 +93,10 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_muon_update.argtypes = [DP, P, P, I, F, P, P]
     lib.ttt_layer.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
     lib.ttt_layer_host.argtypes = [DP, P, P, P, P, P, F, I, P, P, P, S, P]
+    lib.ttt_attention.argtypes = [DP, P, P, P, P, P, P, P, F, I, I, P, P, P, S, P]
+    L64 = ctypes.c_int64
+    lib.ttt_gemm_bf16.argtypes = [I, I, I, P, L64, I, P, L64, I, P, L64, P]
+    lib.ttt_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.ttt_check_status.argtypes = [P, P]
     lib.ttt_status_str.argtypes = [I]
     lib.ttt_status_str.restype = ctypes.c_char_p
@@ -104,7 +110,8 @@ def load_library() -> ctypes.CDLL:
     lib.ttt_kernel_name.restype = ctypes.c_char_p
     for f in ("ttt_shortconv2d", "ttt_write", "ttt_read", "ttt_layer", "ttt_layer_host", "ttt_check_status",
               "ttt_profile_start", "ttt_profile_stop", "ttt_grad", "ttt_sgd_update", "ttt_write_muon",
-              "ttt_layer_muon", "ttt_grad_dot", "ttt_muon_update"):
+              "ttt_layer_muon", "ttt_grad_dot", "ttt_muon_update", "ttt_attention", "ttt_gemm_bf16",
+              "ttt_set_wait_limit"):
         getattr(lib, f).restype = I
     _LIB = lib
     return lib
@@ -273,6 +280,44 @@ def layer(Q, K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out=None, 
     return theta_out, O
 
 
+def attention(X, Wq, Wk, Wv, Wo, conv_w, theta0, lr: float, steps: int, dims, inner: int = INNER_SGD,
+              theta_out=None, out=None, workspace=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The attention layer with the TTT layer inside: q = L2(X Wq), k = L2(X Wk), v = X Wv,
+    the layer (inner loop `inner`), out = O Wo.  X, out: bf16 [n, C]; W*: bf16 [C, C].
+    Returns (theta*, out)."""
+    dm = Dims.of(dims)
+    theta_out = torch.empty_like(theta0) if theta_out is None else theta_out
+    out = torch.empty_like(X) if out is None else out
+    ws = make_workspace(dm, OP_ATTENTION, X.device) if workspace is None else workspace
+    _check(load_library().ttt_attention(ctypes.byref(dm), _dev(X, torch.bfloat16, "X"),
+                                        _dev(Wq, torch.bfloat16, "Wq"), _dev(Wk, torch.bfloat16, "Wk"),
+                                        _dev(Wv, torch.bfloat16, "Wv"), _dev(Wo, torch.bfloat16, "Wo"),
+                                        _dev(conv_w, torch.float32, "conv_w"), _dev(theta0, torch.float32, "theta0"),
+                                        float(lr), int(steps), int(inner),
+                                        _dev(theta_out, torch.float32, "theta_out"), _dev(out, torch.bfloat16, "out"),
+                                        ws.data_ptr(), ws.numel(), _stream()), "ttt_attention")
+    return theta_out, out
+
+
+def gemm_bf16(A: torch.Tensor, B: torch.Tensor, a_t: bool = False, b_t: bool = False,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """C = op(A) op(B) on the library's tensor-core GEMM; op(X) = X.T when the flag is set
+    (the tensor then holds the transpose).  bf16 in and out, FP32 accumulation."""
+    for t, nm in ((A, "A"), (B, "B")):
+        if t.dim() != 2:
+            raise ValueError(f"{nm} must be 2-D")
+    M, K = (A.shape[1], A.shape[0]) if a_t else (A.shape[0], A.shape[1])
+    K2, N = (B.shape[1], B.shape[0]) if b_t else (B.shape[0], B.shape[1])
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
+    _check(load_library().ttt_gemm_bf16(M, N, K, _dev(A, torch.bfloat16, "A"), A.shape[1], int(a_t),
+                                        _dev(B, torch.bfloat16, "B"), B.shape[1], int(b_t),
+                                        _dev(out, torch.bfloat16, "out"), out.shape[1], _stream()),
+           "ttt_gemm_bf16")
+    return out
+
+
 def _host(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
     if t.is_cuda or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous host tensor of {dtype}")
@@ -294,6 +339,11 @@ def layer_host(Q, K, V, conv_w, theta0, lr: float, steps: int, dims, theta_out, 
 def check_status(workspace: torch.Tensor) -> int:
     """Synchronise the current stream and return the workspace's device status (0 = ok)."""
     return int(load_library().ttt_check_status(ctypes.c_void_p(workspace.data_ptr()), _stream()))
+
+
+def set_wait_limit(clocks: int) -> None:
+    """Limit (SM clocks) of every bounded wait in kernels launched from now on; 0 = built-in."""
+    _check(load_library().ttt_set_wait_limit(int(clocks)), "ttt_set_wait_limit")
 
 
 def profile_start() -> None:

@@ -96,3 +96,30 @@ def test_host_validation_codes_of_the_sharded_muon_and_host_entry_points(lib):
     assert lib.ttt_layer_host(dm, None, FAKE, FAKE, FAKE, FAKE, 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
     assert lib.ttt_layer_host(dm, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, -1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
 
+
+
+def test_host_validation_codes_of_the_surround_and_the_gemm(lib):
+    d64 = ctypes.byref(_dims(d=64, h=256, heads=2))
+
+    def att(dm, X=FAKE, inner=0, steps=1):
+        return lib.ttt_attention(dm, X, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, steps, inner, FAKE, FAKE, FAKE,
+                                 1 << 20, None)
+
+    assert att(d64, X=None) == -1
+    assert att(d64, steps=-1) == -1
+    assert att(d64, inner=2) == -1                                   # unknown inner loop
+    assert att(d64, X=FAKE_MIS) == -2
+    assert att(ctypes.byref(_dims(d=32, h=64))) == -3                # heads of 64 only
+    assert att(ctypes.byref(_dims(d=128, h=192))) == -3              # no wide path
+    assert lib.ttt_workspace_bytes(d64, 5) == 0                      # no such op
+
+    def gemm(M=16, N=16, K=16, A=FAKE, lda=16, at=0, ldb=16, bt=0, ldc=16):
+        return lib.ttt_gemm_bf16(M, N, K, A, lda, at, FAKE, ldb, bt, FAKE, ldc, None)
+
+    assert gemm(A=None) == -1
+    assert gemm(M=0) == -1
+    assert gemm(at=2) == -1
+    assert gemm(lda=8) == -1                                         # lda < K
+    assert gemm(N=12, ldb=16, ldc=16) == -2                          # N not a multiple of 8
+    assert gemm(K=20, lda=20, ldb=16) == -2                          # lda not a multiple of 8
+    assert gemm(A=FAKE_MIS) == -2

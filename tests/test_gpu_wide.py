@@ -1,10 +1,12 @@
 """GPU parity of the wide-head path (head widths and hidden widths that are
 multiples of 64 beyond the fused kernels' d <= 64, h <= 256), through the C ABI.
+Every product runs on the library's tensor-core GEMM with the gate, the
+residual and the chain rule in its epilogues.
 
 * Two 128-wide heads with h=192 on a ragged grid: full oracle parity.
 * The 2000-view workload's shape (one head, d=1024, h=2048, lr 0.02, 2 steps)
   on a 4-view subset: full oracle parity.
-* 200 views of that shape (three 131072-token GEMM chunks): the chunk
+* 200 views of that shape (two GEMM chunks of up to 262144 tokens): the chunk
   accumulation checked by the Eq. 5 property delta(all) = sum_parts
   (n_part/n) delta(part) at a step size where one step is far above the f32
   resolution of theta, and bitwise determinism.
@@ -54,7 +56,7 @@ def test_views2000_shape_on_a_view_subset_matches_oracle():
 def test_wide_chunk_accumulation_linearity_and_determinism():
     """One SGD step is delta = -lr grad L(theta0), linear in lr; at lr = 20 the
     step is far above the f32 resolution of theta, so the check isolates the
-    GEMM chunking (three chunks over 200 views, one or two over each part)."""
+    GEMM chunking (two chunks over 200 views, one over each part)."""
     cfg = tin.LayerConfig(BIG.name, 200, BIG.grid_h, BIG.grid_w, BIG.n_special, 1, 1024, 2048, 1, 20.0, BIG.seed)
     inp = tin.make_inputs(cfg, device="cuda")
     K = inp["K"].to(torch.bfloat16).contiguous()

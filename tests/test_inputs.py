@@ -135,3 +135,19 @@ def test_pack_unpack_round_trip(draw):
     assert th.numel() == tin.theta_numel(SMALL.heads, SMALL.d, SMALL.h)
     for a, b in zip(tin.unpack_theta(th, SMALL.heads, SMALL.d, SMALL.h), (draw["W1"], draw["W3"], draw["W2"])):
         assert torch.equal(a, b)
+
+
+def test_surround_draws():
+    c = SMALL.with_views(2)
+    x = tin.make_surround(c)
+    C = c.heads * c.d
+    assert x["X"].shape == (c.n, C)
+    for k in ("Wq", "Wk", "Wv", "Wo"):
+        assert x[k].shape == (C, C)
+        assert torch.equal(x[k], tin.bf16_round(x[k]))
+        assert abs(float(x[k].std()) * C ** 0.5 - 1.0) < 0.02
+    assert torch.equal(x["X"], tin.bf16_round(x["X"]))
+    assert abs(float(x["X"].std()) - 1.0) < 0.02
+    sub = tin.make_surround(c, views=[1])
+    assert torch.equal(sub["X"], x["X"][c.tokens_per_view:])
+    assert not torch.equal(x["Wq"], x["Wk"])
