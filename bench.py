@@ -314,6 +314,10 @@ def run_ours(args, cfg):
 
         def layer_call(Q_, K_, V_, w_, th0_):
             return sharded.layer_sharded(Q_, K_, V_, w_, th0_, cfg.lr, cfg.steps, cfg, n_total, gather, ops)
+    elif args.inner == "muon":
+        # the pages' own inner loop: dot-product loss, Muon steps at their lr 0.1
+        def layer_call(Q_, K_, V_, w_, th0_):
+            return ttt.layer_muon(Q_, K_, V_, w_, th0_, 0.1, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
     else:
         def layer_call(Q_, K_, V_, w_, th0_):
             return ttt.layer(Q_, K_, V_, w_, th0_, cfg.lr, cfg.steps, cfg, theta_out=theta, O=O, workspace=ws)
@@ -554,6 +558,7 @@ def run_ours(args, cfg):
                        "parallelism": (f"{world} GPUs: one {cfg.n_views * world}-view collection sharded by views "
                                        f"({cfg.n_views} per GPU), gradient all-gather per step (NCCL)" if shard
                                        else f"{world} independent replicas" if world > 1 else "1 GPU"),
+                       **({"inner": "dot-product loss + Muon steps, lr 0.1"} if args.inner == "muon" else {}),
                        **({"heldout_views": cfg.heldout_views, "tokens_read": n_read,
                            "value_counts": "the layer's tokens (the held-out read is extra work in each step)"}
                           if cfg.heldout_views else {})},
@@ -603,11 +608,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--views", type=int, default=0,
+                    help="run the workload's shape on this many views instead (small cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the view-count sweep and write/read split")
     ap.add_argument("--no-surround", action="store_true", help="skip the attention-surround measurement")
+    ap.add_argument("--inner", default="sgd", choices=["sgd", "muon"],
+                    help="inner loop of the timed layer: mean-squared loss + SGD, or dot-product loss + Muon")
     ap.add_argument("--replicas", action="store_true",
                     help="with N > 1: independent scenes per GPU instead of one collection sharded by views")
     ap.add_argument("--shard", action="store_true",
@@ -615,6 +624,10 @@ def main():
     args = ap.parse_args()
     from test_layer_reconstruction_b200 import inputs as tin
     cfg = tin.CONFIGS[args.config]
+    if args.views > 0:
+        import dataclasses
+        cfg = dataclasses.replace(cfg.with_views(args.views), name=f"{cfg.name}@{args.views}views",
+                                  heldout_views=min(cfg.heldout_views, args.views))
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -34,8 +34,10 @@ def _until_device_fault(call, ws, attempts=6):
         ttt.set_wait_limit(0)
 
 
+# The wide case uses the 2000-view workload's head (d = 1024, h = 2048) on 4
+# views, so a GEMM tile's accumulation takes microseconds and its waits run out.
 @pytest.mark.parametrize("cfg", [tin.LayerConfig("abort_fused", 6, 37, 37, 5, 4, 64, 256, 2, 0.1, 41),
-                                 tin.LayerConfig("abort_wide", 3, 9, 11, 2, 2, 128, 192, 2, 0.1, 42)],
+                                 tin.CONFIGS["views2000_37x37p5_h1_d1024_h2048"].with_views(4)],
                          ids=["fused", "wide"])
 def test_wait_runs_out_then_the_next_call_succeeds(cfg):
     inp = bf16_inputs(tin.make_inputs(cfg))
