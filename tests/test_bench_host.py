@@ -19,8 +19,8 @@ def test_traffic_digests_match_the_current_sources():
 
 def test_traffic_is_withheld_for_another_workload_or_unknown_kernel():
     t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-    some = next(iter(t["kernels"]))
-    assert bench._traffic_from_profiles(some, "another_workload") is None
+    for some in t["kernels"]:
+        assert bench._traffic_from_profiles(some, "another_workload") is None
     assert bench._traffic_from_profiles("no_such_kernel", t["workload"]) is None
 
 
