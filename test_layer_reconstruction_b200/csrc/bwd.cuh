@@ -17,7 +17,7 @@
 //   Z3^T = W3^T K^T      A = the slice's W3^T rows in shared memory (SS)
 //   dA^T = W2 E^T        A = the slice's W2 rows in shared memory (SS)
 // The epilogue thread of hidden unit r evaluates the chain rule for 16 tokens
-// and writes 2*dZ1^T, dZ3^T and A^T back to TMEM as packed bf16 (2 dZ1^T and
+// and writes 2*dZ1^T, dZ3^T and A^T back to TMEM as packed f16 (2 dZ1^T and
 // dZ3^T over the U columns it has just read, A^T into a small ring); that is
 // exactly the A operand layout of
 //   dW1^T += (2 dZ1^T) K, dW3^T += dZ3^T K, dW2 += A^T E   (M=128 hidden, N=d,
@@ -50,6 +50,7 @@ constexpr int kUnit = 48;             // tokens per backward unit (N of the U/Z3
 constexpr int kBwdThreads = 512;      // 16 warps
 constexpr int kBwdZWarp = 1;
 constexpr int kBwdDwWarp = 2;
+constexpr int kBwdCvtWarp = 3;
 constexpr int kBwdEpiWarp0 = 4;
 constexpr int kBwdStages = 6;         // K/E ring depth
 constexpr int kBwdUBufs = 3;          // U^T buffers
@@ -57,7 +58,7 @@ constexpr int kBwdPaSlots = 2;        // A^T slots
 
 struct BwdParams {
   // Per head, per hidden row r < HIDP: [W1^T row / 2 | W3^T row | W2 row], D
-  // bf16 each (zero for r >= h); read as pairs (element 2c in the low half).
+  // f16 each (zero for r >= h); read as pairs (element 2c in the low half).
   const uint32_t* wt_img;
   float* partials;               // [head*slices+slice][max_contrib][3][128][D] f32
   int n, heads, units, slices;   // units = ceil(n / kUnit); slices = HIDP / 128
@@ -77,7 +78,7 @@ struct BwdLayout {
   static constexpr uint32_t off_k = off_w2 + kWRows;
   static constexpr uint32_t off_e = off_k + kBwdStages * kStage;
   static constexpr uint32_t off_bar = off_e + kBwdStages * kStage;
-  static constexpr int kNumBars = 40;
+  static constexpr int kNumBars = 48;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
   // TMEM columns
   static constexpr uint32_t cW1 = 0;                          // W1^T/2 rows: D/2 columns
@@ -90,11 +91,18 @@ struct BwdLayout {
 };
 
 enum BwdBar {
-  BB_KE_FULL = 0, BB_KE_EMPTY = kBwdStages, BB_W_FULL = 2 * kBwdStages, BB_W_EMPTY, BB_FULL,
+  BB_KE_FULL = 0, BB_KC_FULL = kBwdStages, BB_KE_EMPTY = 2 * kBwdStages, BB_W_FULL = 3 * kBwdStages, BB_W_EMPTY, BB_FULL,
   BB_U_EMPTY = BB_FULL + kBwdUBufs, BB_ZD_EMPTY = BB_U_EMPTY + kBwdUBufs, BB_P_FULL,
   BB_PA_EMPTY = BB_P_FULL + 3 * kBwdUBufs, BB_ACC_FULL = BB_PA_EMPTY + kBwdPaSlots, BB_ACC_EMPTY, BB_DONE
 };
-static_assert(BB_DONE < 40, "barrier count");
+static_assert(BB_DONE < 48, "barrier count");
+
+constexpr uint32_t kHalf2One = 0x3C003C00u;   // (1, 1) in f16x2
+
+// Two bf16 values (one 32-bit word) -> two f16 values (exact in f16's normal range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16x2(bf16lo(v), bf16hi(v));
+}
 
 // Group (of CTAs) that owns flattened (head, unit) item i under the static
 // partition [floor(g*N/G), floor((g+1)*N/G)).
@@ -130,6 +138,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     *abort_flag = 0;
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(&bars[BB_KE_FULL + s], 1);
+      mbar_init(&bars[BB_KC_FULL + s], 1);
       mbar_init(&bars[BB_KE_EMPTY + s], 1);
     }
     mbar_init(&bars[BB_W_FULL], 12);     // every epilogue warp writes part of the weights
@@ -188,9 +197,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_drain(&bars[BB_KE_FULL + jj % kBwdStages], (jj / kBwdStages) & 1);
       }
     }
+  } else if (warp == kBwdCvtWarp) {
+    // ------------------------------------------------------------ K -> f16
+    // In place over the landed bf16 tile (the swizzle permutes whole 16-byte
+    // chunks, so converting every word keeps the layout), then a
+    // generic-to-async proxy fence before the tensor core reads it.
+    Cursor cu;
+    cu.init(it0, p.units);
+    uint32_t s = 0, ph = 0;
+    for (; cu.it < it1; cu.next(p.units)) {
+      if (!mbar_wait_warp(&bars[BB_KE_FULL + s], ph, ab)) break;
+      const uint32_t base = smem_u32(smem + L::off_k + s * L::kStage);
+#pragma unroll 2
+      for (uint32_t off = lane * 16u; off < L::kBox; off += 32u * 16u) {
+        uint32_t a, b, c, d;
+        ld_shared_v4(base + off, a, b, c, d);
+        st_shared_v4(base + off, bf16x2_to_f16x2(a), bf16x2_to_f16x2(b), bf16x2_to_f16x2(c), bf16x2_to_f16x2(d));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BB_KC_FULL + s]);
+      if (++s == kBwdStages) {
+        s = 0;
+        ph ^= 1;
+      }
+    }
   } else if (warp == kBwdZWarp) {
     // ------------------------------------------------------------ U / Z3 / dA issuer
-    constexpr uint32_t kId = idesc_bf16(128, kUnit, false, false);
+    constexpr uint32_t kId = idesc_f16(128, kUnit, false, false);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
     const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
     const uint64_t dw3 = smem_desc(smem_u32(smem + L::off_w3), 0, 8 * SW, SW);
@@ -212,7 +246,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         cur_head = zc.major;
       }
       TTT_TR_LAP(0);
-      if (!(ok = mbar_wait_warp(&bars[BB_KE_FULL + s], ph, ab))) break;
+      if (!(ok = mbar_wait_warp(&bars[BB_KC_FULL + s], ph, ab))) break;
       TTT_TR_LAP(1);
       const uint64_t soff = (s * L::kStage) >> 4;
       const uint64_t dk = dk0 + soff, de = de0 + soff;
@@ -253,7 +287,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // commits release its U buffer, its A^T slot and its K/E stage: the unit's
     // other MMAs completed before the epilogue could read their results, so
     // every reader of the stage is done.
-    constexpr uint32_t kIdW = idesc_bf16(128, D, false, true);
+    constexpr uint32_t kIdW = idesc_f16(128, D, false, true);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::off_k), 0, 8 * SW, SW);
     const uint64_t de0 = smem_desc(smem_u32(smem + L::off_e), 0, 8 * SW, SW);
     const uint32_t tDW = tbase + L::cDW;
@@ -421,21 +455,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t pz1[8], pz3[8], pav[8];
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
-        // Packed bf16 arithmetic on two tokens of this hidden unit (the outputs
-        // are the bf16 A operands of the dW MMAs), with u = z1/2, t = tanh(u):
+        // Packed f16 arithmetic on two tokens of this hidden unit (the outputs
+        // are the f16 A operands of the dW MMAs), with u = z1/2, t = tanh(u):
         //   silu = u (1+t),  2 dsilu/dz1 = (1+t) + u (1 - t^2),
         //   2 dZ1 = dA z3 (2 dsilu/dz1),  dZ3 = dA silu,  A = silu z3.
-        const uint32_t bu = pack_bf16x2(__uint_as_float(zu[i]), __uint_as_float(zu[i + 1]));
-        const uint32_t b3 = pack_bf16x2(__uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
-        const uint32_t bd = pack_bf16x2(__uint_as_float(da[i]), __uint_as_float(da[i + 1]));
-        const uint32_t t = btanh2(bu);
-        const uint32_t s2 = bfma2(t, kBf2One, kBf2One);                 // 1 + t
-        const uint32_t silu = bmul2(bu, s2);
-        const uint32_t om = bfma2(t ^ 0x80008000u, t, kBf2One);          // 1 - t^2
-        const uint32_t q2 = bfma2(bu, om, s2);                          // 2 dsilu/dz1
-        pz1[i / 2] = bmul2(bmul2(bd, b3), q2);
-        pz3[i / 2] = bmul2(bd, silu);
-        pav[i / 2] = bmul2(silu, b3);
+        const uint32_t bu = pack_f16x2(__uint_as_float(zu[i]), __uint_as_float(zu[i + 1]));
+        const uint32_t b3 = pack_f16x2(__uint_as_float(z3[i]), __uint_as_float(z3[i + 1]));
+        const uint32_t bd = pack_f16x2(__uint_as_float(da[i]), __uint_as_float(da[i + 1]));
+        const uint32_t t = htanh2(bu);
+        const uint32_t s2 = hfma2(t, kHalf2One, kHalf2One);              // 1 + t
+        const uint32_t silu = hmul2(bu, s2);
+        const uint32_t om = hfma2(t ^ 0x80008000u, t, kHalf2One);         // 1 - t^2
+        const uint32_t q2 = hfma2(bu, om, s2);                          // 2 dsilu/dz1
+        pz1[i / 2] = hmul2(hmul2(bd, b3), q2);
+        pz3[i / 2] = hmul2(bd, silu);
+        pav[i / 2] = hmul2(silu, b3);
       }
       TTT_TR_LAP(3);
       // 2 dZ1^T, dZ3^T over this warpgroup's U columns (read above); A^T into

@@ -4,7 +4,8 @@
 // sequence to (N, H/p, W/p, d), convolve with a 3x3 filter, flatten; the
 // convolution stays inside one image; camera and register tokens pass through
 // unmixed, Appendix A).  Cross-correlation with zero padding, no bias,
-// FP32 accumulation, bf16 round-to-nearest-even store.
+// FP32 accumulation, bf16 round-to-nearest-even store (or f16 for the
+// backward kernel's operand in the dot-product-loss path).
 //
 // HBM-bound: every value is read once from DRAM and V' written once.  A
 // thread owns 4 channels (one 8-byte vector) of a band of kConvBand grid rows
@@ -57,6 +58,15 @@ __device__ __forceinline__ uint32_t bf16x2_from_f32x2(uint64_t v) {
   asm("{ .reg .b32 l, h; mov.b64 {l, h}, %1; cvt.rn.bf16x2.f32 %0, h, l; }" : "=r"(r) : "l"(v));
   return r;
 }
+__device__ __forceinline__ uint32_t f16x2_from_f32x2(uint64_t v) {
+  uint32_t r;
+  asm("{ .reg .b32 l, h; mov.b64 {l, h}, %1; cvt.rn.f16x2.f32 %0, h, l; }" : "=r"(r) : "l"(v));
+  return r;
+}
+// Two bf16 values -> two f16 values (rounded to nearest; exact in f16's normal range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_exact(uint32_t v) {
+  return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
 
 constexpr int kConvRing = 8;   // columns in the per-thread shared-memory ring
 constexpr int kConvBand = 3;   // output rows per thread
@@ -81,7 +91,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Block b walks the items b, b + gridDim.x, ... of the (view, band) space,
 // band == bands meaning the view's special tokens.  A thread's 36 weights are
 // loaded once per block instead of once per band.
-template <int R>
+template <int R, bool F16OUT>
 __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvParams p) {
   constexpr int NR = R + 2;   // input rows of a band
   extern __shared__ __align__(16) uint8_t conv_smem[];
@@ -110,7 +120,8 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
     if (band == bands) {
       for (int s = 0; s < p.n_special; ++s) {
         const long long t = vbase + s;
-        p.out[t * G4 + cg] = __ldg(p.V + t * G4 + cg);
+        const uint2 v = __ldg(p.V + t * G4 + cg);
+        p.out[t * G4 + cg] = F16OUT ? make_uint2(bf16x2_to_f16x2_exact(v.x), bf16x2_to_f16x2_exact(v.y)) : v;
       }
       continue;
     }
@@ -179,8 +190,9 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
             f32x2_fma(acc[q], wp[q][3 * a + 2], Rt[r + a][q]);
           }
         if (out_ok[r])
-          outp[r * out_row + static_cast<long long>(x) * G4] = make_uint2(bf16x2_from_f32x2(acc[0]),
-                                                                          bf16x2_from_f32x2(acc[1]));
+          outp[r * out_row + static_cast<long long>(x) * G4] =
+              F16OUT ? make_uint2(f16x2_from_f32x2(acc[0]), f16x2_from_f32x2(acc[1]))
+                     : make_uint2(bf16x2_from_f32x2(acc[0]), bf16x2_from_f32x2(acc[1]));
       }
       cp_async_wait<kConvRing - 3>();
       take(x + 2, L);

@@ -4,7 +4,7 @@
 // (VGG-T$^3$: Offline Feed-Forward 3D Reconstruction at Scale, Sec. 3.4,
 // Eq. 4 and "TTT MLP Architecture and Inner Optimization").
 //   READ mode : X = Q, writes O = Y (bf16).
-//   WRITE mode: X = K, writes the residual E = Y - V' (bf16); the backward
+//   WRITE mode: X = K, writes the residual E = Y - V' (f16); the backward
 //               kernel turns it into the gradient, the factor 2/n of the
 //               mean-squared loss is applied in the update.
 //
@@ -42,7 +42,7 @@ constexpr int kPrefetchAhead = 3;    // items whose tiles the producer prefetche
 struct FwdParams {
   const __nv_bfloat16* w13_img;  // per head: 2*HIDP rows of D bf16 (sw-swizzled)
   const __half* w2_img;          // per head: HIDP rows of D f16 (sw-swizzled)
-  __nv_bfloat16* out;            // [n][heads][D]
+  __nv_bfloat16* out;            // [n][heads][D]: O (bf16) or, in WRITE mode, E (f16 bits)
   int n, heads, tiles;
   unsigned int* status;
   long long wait_clocks;         // limit of a bounded wait (<= 0: the default)
@@ -374,13 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long tok = static_cast<long long>(tile) * kTileM + row;
       if (tok < p.n) {
         uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + head) * D + hf * kYHalf);
+        // O in bf16; the residual E in f16, the backward kernel's operand type
+        auto pk = [](float a, float b) { return WRITE ? pack_f16x2(a, b) : pack_bf16x2(a, b); };
 #pragma unroll
         for (int ch = 0; ch < kYHalf / 8; ++ch) {
           uint4 v;
-          v.x = pack_bf16x2(y[8 * ch + 0], y[8 * ch + 1]);
-          v.y = pack_bf16x2(y[8 * ch + 2], y[8 * ch + 3]);
-          v.z = pack_bf16x2(y[8 * ch + 4], y[8 * ch + 5]);
-          v.w = pack_bf16x2(y[8 * ch + 6], y[8 * ch + 7]);
+          v.x = pk(y[8 * ch + 0], y[8 * ch + 1]);
+          v.y = pk(y[8 * ch + 2], y[8 * ch + 3]);
+          v.z = pk(y[8 * ch + 4], y[8 * ch + 5]);
+          v.w = pk(y[8 * ch + 6], y[8 * ch + 7]);
           dst[ch] = v;
         }
       }

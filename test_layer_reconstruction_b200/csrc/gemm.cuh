@@ -14,19 +14,28 @@
 //             [M][K], B stored [N][K]); TMA box 64 (K) x 128 rows.
 //   MN-major: the rows are K and M (or N) is contiguous (A stored [K][M],
 //             B stored [K][N]); TMA box 64 (M or N) x 64 (K rows).
-// Both use the 128-byte swizzle.  Tiles are 128 x 256 (M x N) with K steps
-// of 64: per stage one or two A boxes (16 KiB) and two or four B boxes
-// (32 KiB), four stages.  Each k step issues four M=128, N=256, K=16 MMAs;
-// at that shape an SS MMA reads 96 B/clk of shared memory, under the ~128
-// B/clk the tensor core takes, so it runs at full rate.
+// Both use the 128-byte swizzle.
 //
-// One persistent CTA per SM walks the work items (problem, M tile, N tile,
-// K split) of up to three problems with a static stride.  Warp roles:
+// CTA pairs (clusters of two) share each 256 x 256 tile through the
+// tensor cores' two-CTA form (cta_group::2): CTA r of the pair loads rows
+// 128r..128r+127 of the tile's A and columns 128r..128r+127 of its B (16 KiB
+// each per K step of 64), the leader issues M=256, N=256, K=16 MMAs that read
+// both CTAs' shared memory, and each CTA's tensor memory holds its own 128
+// rows of the accumulator.  Per SM and K step that is 32 KiB of operands for
+// 2 x 128 x 256 x 64 FLOPs, a third less than a one-CTA 128 x 256 tile, which
+// leaves shared-memory bandwidth for the epilogue and fits six stages.  Both
+// CTAs' loads complete on the leader's stage barrier; the leader's commits
+// reach both CTAs' barriers (multicast to the pair); each CTA's epilogue
+// arrives on the leader's accumulator-free barrier.
+//
+// Each pair walks the work items (problem, 256-row M tile, N tile, K split)
+// of up to three problems with a static stride.  Warp roles, in both CTAs:
 //   warp 0     TMA producer
-//   warp 1     TMEM allocator and MMA issuer (warp-uniform, one elected lane)
+//   warp 1     TMEM allocator; in the leader also the MMA issuer
+//              (warp-uniform, one elected lane)
 //   warps 4-11 epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (rows of
-//              the tile); warps 4-7 take the first half of the tile's
-//              columns, warps 8-11 the second.
+//              the CTA's half tile); warps 4-7 take the first half of the
+//              tile's columns, warps 8-11 the second.
 // The accumulator is double buffered in TMEM (2 x 256 columns), so the
 // epilogue of one tile overlaps the MMAs of the next.  Rows and columns past
 // a problem's M and N are computed on TMA's zero fill and not stored.
@@ -54,8 +63,9 @@
 
 namespace ttt {
 
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kGemmBM = 256, kGemmBN = 256, kGemmBK = 64;   // tile of a CTA pair
+constexpr int kGemmHalfM = kGemmBM / 2, kGemmHalfN = kGemmBN / 2; // loaded by each CTA
+constexpr int kGemmStages = 6;
 constexpr int kGemmThreads = 384;    // 12 warps
 constexpr int kGemmEpiWarp0 = 4;
 constexpr int kGemmMaxProblems = 3;
@@ -96,8 +106,8 @@ struct GemmParams {
 };
 
 struct GemmLayout {
-  static constexpr uint32_t kA = kGemmBM * kGemmBK * 2;   // 16 KiB
-  static constexpr uint32_t kB = kGemmBN * kGemmBK * 2;   // 32 KiB
+  static constexpr uint32_t kA = kGemmHalfM * kGemmBK * 2;   // 16 KiB: this CTA's A rows
+  static constexpr uint32_t kB = kGemmHalfN * kGemmBK * 2;   // 16 KiB: this CTA's B columns
   static constexpr uint32_t kStage = kA + kB;
   static constexpr uint32_t off_bar = kGemmStages * kStage;
   static constexpr int kNumBars = 2 * kGemmStages + 4 + 1;
@@ -136,6 +146,68 @@ __device__ __forceinline__ void gemm_k_range(const GemmProblem& q, int s, int* k
 
 __device__ __forceinline__ uint32_t gemm_idesc(int a_mn, int b_mn) {
   return idesc_bf16(kGemmBM, kGemmBN, a_mn != 0, b_mn != 0);
+}
+
+// ------------------------------------------------------------------ CTA pairs
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier given by its cluster address (this CTA's or the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem, both CTAs] (+)= A[smem, both CTAs] * B[smem, both CTAs], issued by one elected lane.
+__device__ __forceinline__ void mma_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this address in both CTAs of the pair when
+// every MMA issued so far by this thread completes.
+__device__ __forceinline__ void mma_commit_pair_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
 }
 
 // 32 lanes x 32 bits, 32 consecutive columns per thread.
@@ -188,31 +260,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const Abort ab{abort_flag, P.status, P.wait_clocks};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();           // 0: the pair's leader
+  const long long pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < kGemmStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1);     // the leader's expect_tx; both CTAs' loads complete on it
+      mbar_init(&empty[s], 1);    // the leader's commit, multicast to both CTAs
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);
+      mbar_init(&acc_empty[b], 16);   // the epilogue warps of both CTAs (the leader's is used)
     }
     mbar_init(done, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // both CTAs' barriers exist before either CTA signals the other's
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       const CUtensorMap* ma[3] = {&tma0, &tma1, &tma2};
       const CUtensorMap* mb[3] = {&tmb0, &tmb1, &tmb2};
@@ -220,33 +295,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_prefetch_desc(ma[p]);
         tma_prefetch_desc(mb[p]);
       }
+      const uint32_t full_leader = map_to_rank(smem_u32(full), 0);
       uint32_t stage = 0, ph = 0, issued = 0;
       bool ok = true;
-      for (long long it = blockIdx.x; it < P.total_items && ok; it += gridDim.x) {
+      for (long long it = pair; it < P.total_items && ok; it += npairs) {
         const GemmItem w = gemm_item(P, it);
         const GemmProblem& q = P.prob[w.p];
         int k0, nkb;
         gemm_k_range(q, w.s, &k0, &nkb);
-        const int m0 = w.tm * kGemmBM, n0 = w.tn * kGemmBN;
+        const int m0 = w.tm * kGemmBM + rank * kGemmHalfM, n0 = w.tn * kGemmBN + rank * kGemmHalfN;
         for (int kb = 0; kb < nkb; ++kb) {
           const int k = k0 + kb * kGemmBK;
           if (!(ok = mbar_wait(&empty[stage], ph ^ 1, ab))) break;
-          mbar_arrive_expect_tx(&full[stage], L::kStage);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStage);
+          const uint32_t bar = full_leader + stage * 8;
           uint8_t* sa = smem + stage * L::kStage;
           uint8_t* sb = sa + L::kA;
           if (q.a_mn) {
-            tma_load_2d(sa, ma[w.p], &full[stage], q.a_x0 + m0, q.a_y0 + k);
-            tma_load_2d(sa + 8192, ma[w.p], &full[stage], q.a_x0 + m0 + 64, q.a_y0 + k);
+            tma_load_2d_pair(sa, ma[w.p], bar, q.a_x0 + m0, q.a_y0 + k);
+            tma_load_2d_pair(sa + 8192, ma[w.p], bar, q.a_x0 + m0 + 64, q.a_y0 + k);
           } else {
-            tma_load_2d(sa, ma[w.p], &full[stage], q.a_x0 + k, q.a_y0 + m0);
+            tma_load_2d_pair(sa, ma[w.p], bar, q.a_x0 + k, q.a_y0 + m0);
           }
           if (q.b_mn) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              tma_load_2d(sb + i * 8192, mb[w.p], &full[stage], q.b_x0 + n0 + 64 * i, q.b_y0 + k);
+            tma_load_2d_pair(sb, mb[w.p], bar, q.b_x0 + n0, q.b_y0 + k);
+            tma_load_2d_pair(sb + 8192, mb[w.p], bar, q.b_x0 + n0 + 64, q.b_y0 + k);
           } else {
-            tma_load_2d(sb, mb[w.p], &full[stage], q.b_x0 + k, q.b_y0 + n0);
-            tma_load_2d(sb + 16384, mb[w.p], &full[stage], q.b_x0 + k, q.b_y0 + n0 + 128);
+            tma_load_2d_pair(sb, mb[w.p], bar, q.b_x0 + k, q.b_y0 + n0);
           }
           ++issued;
           if (++stage == kGemmStages) {
@@ -255,67 +330,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // Drain: the last load issued into each stage has landed before exit.
-      const uint32_t last = issued < static_cast<uint32_t>(kGemmStages) ? issued : kGemmStages;
-      for (uint32_t b = 0; b < last; ++b) {
-        const uint32_t jj = issued - 1 - b;
-        mbar_drain(&full[jj % kGemmStages], (jj / kGemmStages) & 1);
+      // Drain (leader): the stage barriers count both CTAs' loads, so the last
+      // load issued into each stage by either CTA has landed before exit.  The
+      // peer cannot wait on the leader's barriers; it leaves only after the
+      // closing cluster barrier, which the leader reaches after this drain.
+      if (rank == 0) {
+        const uint32_t last = issued < static_cast<uint32_t>(kGemmStages) ? issued : kGemmStages;
+        for (uint32_t b = 0; b < last; ++b) {
+          const uint32_t jj = issued - 1 - b;
+          mbar_drain(&full[jj % kGemmStages], (jj / kGemmStages) & 1);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t sbase = smem_u32(smem);
-    uint32_t stage = 0, ph = 0, local = 0;
-    bool ok = true;
-    for (long long it = blockIdx.x; it < P.total_items && ok; it += gridDim.x, ++local) {
-      const GemmItem w = gemm_item(P, it);
-      const GemmProblem& q = P.prob[w.p];
-      int k0, nkb;
-      gemm_k_range(q, w.s, &k0, &nkb);
-      const uint32_t buf = local & 1;
-      if (!(ok = mbar_wait_warp(&acc_empty[buf], ((local >> 1) & 1) ^ 1, ab))) break;
-      tc_fence_after();
-      const uint32_t idesc = gemm_idesc(q.a_mn, q.b_mn);
-      // per K=16 step: K-major operands advance 32 bytes, MN-major ones 16 rows of 128 bytes
-      const uint32_t a_step = q.a_mn ? 2048u : 32u, b_step = q.b_mn ? 2048u : 32u;
-      const uint32_t a_lbo = q.a_mn ? 8192u : 16u, b_lbo = q.b_mn ? 8192u : 16u;
-      const uint32_t tacc = tbase + buf * kGemmBN;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!(ok = mbar_wait_warp(&full[stage], ph, ab))) break;
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (rank == 0) {
+      const uint32_t sbase = smem_u32(smem);
+      uint32_t stage = 0, ph = 0, local = 0;
+      bool ok = true;
+      for (long long it = pair; it < P.total_items && ok; it += npairs, ++local) {
+        const GemmItem w = gemm_item(P, it);
+        const GemmProblem& q = P.prob[w.p];
+        int k0, nkb;
+        gemm_k_range(q, w.s, &k0, &nkb);
+        const uint32_t buf = local & 1;
+        if (!(ok = mbar_wait_warp(&acc_empty[buf], ((local >> 1) & 1) ^ 1, ab))) break;
         tc_fence_after();
-        const uint32_t sa = sbase + stage * L::kStage, sb = sa + L::kA;
-        const uint64_t ad = smem_desc(sa, a_lbo, 1024, 128), bd = smem_desc(sb, b_lbo, 1024, 128);
+        const uint32_t idesc = gemm_idesc(q.a_mn, q.b_mn);
+        // per K=16 step: K-major operands advance 32 bytes, MN-major ones 16 rows of 128 bytes
+        const uint32_t a_step = q.a_mn ? 2048u : 32u, b_step = q.b_mn ? 2048u : 32u;
+        const uint32_t a_lbo = q.a_mn ? 8192u : 16u, b_lbo = q.b_mn ? 8192u : 16u;
+        const uint32_t tacc = tbase + buf * kGemmBN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!(ok = mbar_wait_warp(&full[stage], ph, ab))) break;
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::kStage, sb = sa + L::kA;
+          const uint64_t ad = smem_desc(sa, a_lbo, 1024, 128), bd = smem_desc(sb, b_lbo, 1024, 128);
 #pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k)
-          mma_bf16_warp(tacc, ad + ((k * a_step) >> 4), bd + ((k * b_step) >> 4), idesc,
-                        (kb > 0 || k > 0) ? 1u : 0u);
-        mma_commit_warp(&empty[stage]);
-        if (++stage == kGemmStages) {
-          stage = 0;
-          ph ^= 1;
+          for (int k = 0; k < kGemmBK / 16; ++k)
+            mma_pair_warp(tacc, ad + ((k * a_step) >> 4), bd + ((k * b_step) >> 4), idesc,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit_pair_warp(&empty[stage]);
+          if (++stage == kGemmStages) {
+            stage = 0;
+            ph ^= 1;
+          }
         }
+        if (ok) mma_commit_pair_warp(&acc_full[buf]);
       }
-      if (ok) mma_commit_warp(&acc_full[buf]);
+      // All issued MMAs (which write both CTAs' tensor memory) have completed
+      // before either CTA releases it.
+      mma_commit_pair_warp(done);
     }
-    // All issued MMAs have completed before TMEM is released.
-    mma_commit_warp(done);
     mbar_drain(done, 0);
   } else if (warp >= kGemmEpiWarp0) {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int e = warp - kGemmEpiWarp0;      // 0..7
     const int quad = warp & 3;               // TMEM lane quadrant
     const int hf = e >> 2;                   // column half of the tile
-    const int row = quad * 32 + lane;        // row of the tile
+    const int row = quad * 32 + lane;        // row of this CTA's half tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
     uint32_t local = 0;
-    for (long long it = blockIdx.x; it < P.total_items; it += gridDim.x, ++local) {
+    for (long long it = pair; it < P.total_items; it += npairs, ++local) {
       const GemmItem w = gemm_item(P, it);
       const GemmProblem& q = P.prob[w.p];
       const uint32_t buf = local & 1;
       if (!mbar_wait_warp(&acc_full[buf], (local >> 1) & 1, ab)) break;
       tc_fence_after();
       const uint32_t tacc = tbase + buf * kGemmBN + lane_off;
-      const long long m = static_cast<long long>(w.tm) * kGemmBM + row;
+      const long long m = static_cast<long long>(w.tm) * kGemmBM + rank * kGemmHalfM + row;
       const bool row_ok = m < q.M;
       const int n0 = w.tn * kGemmBN;
       if (EPI == kEpiGate) {
@@ -452,15 +536,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader + buf * 8);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // no signal to the peer is still on its way, and no MMA writes TMEM
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 512);
+    tmem_dealloc_pair(tbase, 512);
   }
 }
 

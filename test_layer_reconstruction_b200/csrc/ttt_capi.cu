@@ -262,8 +262,10 @@ bool aligned(const void* p, size_t a = 16) { return (reinterpret_cast<uintptr_t>
 int launch_status() { return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ECUDA; }
 
 // ------------------------------------------------------------------ launches
+// V' = ShortConv2D(V), stored as bf16, or as f16 with `f16out` (the
+// backward kernel's operand type, for the dot-product-loss path).
 int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float* w, uint16_t* out,
-             cudaStream_t st) {
+             cudaStream_t st, bool f16out = false) {
   ConvParams p;
   p.V = reinterpret_cast<const uint2*>(V);
   p.w = w;
@@ -280,11 +282,11 @@ int run_conv(const Shape& s, const ttt_dims* dm, const uint16_t* V, const float*
   const long long persistent = static_cast<long long>(sms > 0 ? sms : 148) * 2;
   dim3 grid(static_cast<unsigned>(std::min(items, persistent)), (g4 + block - 1) / block, 1);
   const size_t smem = conv_smem_bytes(block);
-  if (cudaFuncSetAttribute(shortconv_kernel<kConvBand>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  auto k = f16out ? shortconv_kernel<kConvBand, true> : shortconv_kernel<kConvBand, false>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TTT_ECUDA;
   ProfScope prof(KK_CONV, st);
-  shortconv_kernel<kConvBand><<<grid, block, smem, st>>>(p);
+  k<<<grid, block, smem, st>>>(p);
   return launch_status();
 }
 
@@ -294,7 +296,7 @@ int run_pack(const Shape& s, const float* theta, const Ws& w, uint8_t* ws, bool 
   p.theta = theta;
   p.w13_img = reinterpret_cast<__nv_bfloat16*>(ws + w.w13);
   p.w2h_img = reinterpret_cast<__half*>(ws + w.w2h);
-  p.wt_img = with_wt ? reinterpret_cast<__nv_bfloat16*>(ws + w.wt) : nullptr;
+  p.wt_img = with_wt ? reinterpret_cast<__half*>(ws + w.wt) : nullptr;
   p.heads = s.H;
   p.d = s.D;
   p.h = s.h;
@@ -434,20 +436,34 @@ int launch_gemm(GemmLaunch& g, unsigned int* status, int kind, cudaStream_t st) 
     g.ma[p] = g.ma[0];
     g.mb[p] = g.mb[0];
   }
+  // one CTA pair (a cluster of two) per two SMs
   const int sms = num_sms();
-  const int grid = static_cast<int>(std::min<long long>(sms > 0 ? sms : 148, g.P.total_items));
+  const long long pairs = std::min<long long>((sms > 1 ? sms : 148) / 2, g.P.total_items);
   auto k = gemm_kernel<EPI>;
   const uint32_t smem = GemmLayout::bytes;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return TTT_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   ProfScope prof(kind, st);
-  k<<<grid, kGemmThreads, smem, st>>>(g.ma[0], g.mb[0], g.ma[1], g.mb[1], g.ma[2], g.mb[2], g.P);
+  if (cudaLaunchKernelEx(&cfg, k, g.ma[0], g.mb[0], g.ma[1], g.mb[1], g.ma[2], g.mb[2], g.P) != cudaSuccess)
+    return TTT_ECUDA;
   return launch_status();
 }
 
 // K splits of the weight-gradient launch: enough items for about three waves
-// of one CTA per SM.
+// of one CTA pair per two SMs.
 int wgrad_splits(const Shape& s, long long nc) {
-  const int sms = std::max(1, num_sms());
+  const int sms = std::max(2, num_sms()) / 2;
   const long long tiles = 2LL * ((s.D + kGemmBM - 1) / kGemmBM) * ((s.h + kGemmBN - 1) / kGemmBN) +
                           static_cast<long long>((s.h + kGemmBM - 1) / kGemmBM) * ((s.D + kGemmBN - 1) / kGemmBN);
   const long long want = (3LL * sms + tiles - 1) / tiles;
@@ -799,13 +815,15 @@ int run_muon_update(const Shape& s, const float* theta_in, const float* grads, i
   return launch_status();
 }
 
-// The pages' inner loop: `steps` Muon steps on the dot-product loss.
+// The pages' inner loop: `steps` Muon steps on the dot-product loss.  The
+// gradient's output factor is the constant -V', which the backward kernel
+// reads where it reads E, so V' is stored in f16, its operand type.
 int run_write_muon(const Call& c, const ttt_dims* dm, const uint16_t* K, const uint16_t* V, const float* conv_w,
                    const float* theta0, float lr, int steps, float* theta_out) {
   const Shape& s = c.s;
   uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
   float* grad = reinterpret_cast<float*>(c.ws + c.w.grad);
-  int rc = run_conv(s, dm, V, conv_w, vp, c.st);
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st, true);
   if (rc != TTT_OK) return rc;
   if (steps == 0) {
     if (theta_out != theta0 &&
@@ -1013,8 +1031,14 @@ int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, co
   Call c;
   rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
+  // the backward kernel reads V' in f16, its operand type
+  uint16_t* vp16 = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
+  const long long count = c.s.n * c.s.C;
+  bf16_to_f16_kernel<<<elementwise_grid(count / 8), 256, 0, c.st>>>(reinterpret_cast<const uint4*>(Vp),
+                                                                     reinterpret_cast<uint4*>(vp16), count / 8);
+  if ((rc = launch_status()) != TTT_OK) return rc;
   GradPass gp;
-  if (!setup_grad_pass(c, K, Vp, &gp, true)) return TTT_ECUDA;
+  if (!setup_grad_pass(c, K, vp16, &gp, true)) return TTT_ECUDA;
   return run_grad_pass(c, gp, theta, nullptr, -1.f, grad, true);
 }
 

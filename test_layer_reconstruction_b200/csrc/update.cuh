@@ -23,9 +23,9 @@
 //     sub-chunk s, 32 rows of W1^T (hidden s*32+r) then 32 rows of W3^T.
 //   W2 image (f16, same tiling), per head: row j = W2[j][:]; the forward
 //     kernel's gate operand is f16.
-//   WT image (bf16, plain rows; write path only), per head and hidden unit r:
+//   WT image (f16, plain rows; write path only), per head and hidden unit r:
 //     [W1^T row r / 2 | W3^T row r | W2 row r], the backward kernel's weight
-//     rows (halving is exact in bf16).
+//     rows (halving is exact).
 #pragma once
 #include "bwd.cuh"
 
@@ -84,11 +84,21 @@ __global__ void sgd_sum_kernel(const float* theta_in, const float* __restrict__ 
   }
 }
 
+// bf16 -> f16 (round to nearest; exact in f16's normal range), 8 values per
+// thread and iteration.
+__global__ void bf16_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = src[i];
+    dst[i] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+  }
+}
+
 struct PackParams {
   const float* theta;
   __nv_bfloat16* w13_img;
   __half* w2h_img;
-  __nv_bfloat16* wt_img;  // null: not written
+  __half* wt_img;         // null: not written
   int heads, d, h, hidp;
 };
 
@@ -144,7 +154,7 @@ __global__ void pack_images_kernel(const PackParams p) {
         v = p.theta[2 * hdh + static_cast<size_t>(head) * p.h * D + static_cast<size_t>(r) * D + col];
       }
     }
-    p.wt_img[k] = __float2bfloat16_rn(v);
+    p.wt_img[k] = __float2half_rn(v);
   }
 }
 
