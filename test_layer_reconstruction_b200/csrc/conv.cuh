@@ -4,8 +4,8 @@
 // sequence to (N, H/p, W/p, d), convolve with a 3x3 filter, flatten; the
 // convolution stays inside one image; camera and register tokens pass through
 // unmixed, Appendix A).  Cross-correlation with zero padding, no bias,
-// FP32 accumulation, bf16 round-to-nearest-even store (or f16 for the
-// backward kernel's operand in the dot-product-loss path).
+// FP32 accumulation, bf16 round-to-nearest-even store (widened exactly to
+// f16, the backward kernel's operand type, in the dot-product-loss path).
 //
 // HBM-bound: every value is read once from DRAM and V' written once.  A
 // thread owns 4 channels (one 8-byte vector) of a band of kConvBand grid rows
@@ -56,11 +56,6 @@ __device__ __forceinline__ void f32x2_fma(uint64_t& acc, uint64_t a, uint64_t b)
 __device__ __forceinline__ uint32_t bf16x2_from_f32x2(uint64_t v) {
   uint32_t r;
   asm("{ .reg .b32 l, h; mov.b64 {l, h}, %1; cvt.rn.bf16x2.f32 %0, h, l; }" : "=r"(r) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ uint32_t f16x2_from_f32x2(uint64_t v) {
-  uint32_t r;
-  asm("{ .reg .b32 l, h; mov.b64 {l, h}, %1; cvt.rn.f16x2.f32 %0, h, l; }" : "=r"(r) : "l"(v));
   return r;
 }
 // Two bf16 values -> two f16 values (rounded to nearest; exact in f16's normal range).
@@ -189,10 +184,13 @@ __global__ void __launch_bounds__(kConvThreads, 2) shortconv_kernel(const ConvPa
             f32x2_fma(acc[q], wp[q][3 * a + 1], M[r + a][q]);
             f32x2_fma(acc[q], wp[q][3 * a + 2], Rt[r + a][q]);
           }
-        if (out_ok[r])
+        // f16 output: V' is rounded to bf16 first, as every path stores it, then
+        // widened exactly, so it equals the bf16 output converted to f16.
+        if (out_ok[r]) {
+          const uint2 b = make_uint2(bf16x2_from_f32x2(acc[0]), bf16x2_from_f32x2(acc[1]));
           outp[r * out_row + static_cast<long long>(x) * G4] =
-              F16OUT ? make_uint2(f16x2_from_f32x2(acc[0]), f16x2_from_f32x2(acc[1]))
-                     : make_uint2(bf16x2_from_f32x2(acc[0]), bf16x2_from_f32x2(acc[1]));
+              F16OUT ? make_uint2(bf16x2_to_f16x2_exact(b.x), bf16x2_to_f16x2_exact(b.y)) : b;
+        }
       }
       cp_async_wait<kConvRing - 3>();
       take(x + 2, L);

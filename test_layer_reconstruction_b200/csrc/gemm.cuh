@@ -109,7 +109,10 @@ struct GemmLayout {
   static constexpr uint32_t kA = kGemmHalfM * kGemmBK * 2;   // 16 KiB: this CTA's A rows
   static constexpr uint32_t kB = kGemmHalfN * kGemmBK * 2;   // 16 KiB: this CTA's B columns
   static constexpr uint32_t kStage = kA + kB;
-  static constexpr uint32_t off_bar = kGemmStages * kStage;
+  // per epilogue warp: 32 rows x 64 bytes, rows padded to 80 bytes (no bank conflicts)
+  static constexpr uint32_t kStgPitch = 80, kStgBytes = 32 * kStgPitch;
+  static constexpr uint32_t off_stg = kGemmStages * kStage;
+  static constexpr uint32_t off_bar = off_stg + 8 * kStgBytes;
   static constexpr int kNumBars = 2 * kGemmStages + 4 + 1;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
 };
@@ -235,6 +238,70 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v)
 }
 __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float* v) {
   const uint4 u = *reinterpret_cast<const uint4*>(src);
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x);
+  v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z);
+  v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
+// Coalesced epilogue I/O.  A warp's 32 threads own 32 rows of the tile (one
+// row each, the layout of the tensor-memory loads); written straight to
+// global memory, one instruction would touch 32 rows.  Staged through the
+// warp's 32 x 64-byte shared buffer instead, each instruction moves 64
+// contiguous bytes of 8 rows.  `m0` is the warp's first row; rows at or past
+// `M` and 8-column groups at or past `N` are skipped.
+struct StageIO {
+  uint32_t buf;   // this warp's staging buffer (shared address)
+  int lane;
+  // This thread's 32 bf16 (four 16-byte vectors) of its row -> rows m0.. of
+  // `dst` (row pitch `ld` elements) at column `col`.
+  __device__ __forceinline__ void store_bf16(const uint4 (&v)[4], __nv_bfloat16* dst, long long ld, long long m0,
+                                             long long M, int col, int N) const {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) st_shared_v4(buf + lane * GemmLayout::kStgPitch + c * 16, v[c].x, v[c].y, v[c].z, v[c].w);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + (lane >> 2), c = lane & 3;
+      uint4 x;
+      ld_shared_v4(buf + r * GemmLayout::kStgPitch + c * 16, x.x, x.y, x.z, x.w);
+      if (m0 + r < M && col + 8 * c < N) *reinterpret_cast<uint4*>(dst + (m0 + r) * ld + col + 8 * c) = x;
+    }
+    __syncwarp();
+  }
+  // The reverse: rows m0.. of `src` at column `col` -> this thread's row (32 bf16).
+  __device__ __forceinline__ void load_bf16(uint4 (&v)[4], const __nv_bfloat16* src, long long ld, long long m0,
+                                            long long M, int col, int N) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + (lane >> 2), c = lane & 3;
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (m0 + r < M && col + 8 * c < N) x = *reinterpret_cast<const uint4*>(src + (m0 + r) * ld + col + 8 * c);
+      st_shared_v4(buf + r * GemmLayout::kStgPitch + c * 16, x.x, x.y, x.z, x.w);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ld_shared_v4(buf + lane * GemmLayout::kStgPitch + c * 16, v[c].x, v[c].y, v[c].z, v[c].w);
+    __syncwarp();
+  }
+  // f32 versions: 16 floats (64 bytes) of the row.
+  __device__ __forceinline__ void store_f32(const float4 (&v)[4], float* dst, long long ld, long long m0, long long M,
+                                            int col, int N) const {
+    store_bf16(reinterpret_cast<const uint4(&)[4]>(v), reinterpret_cast<__nv_bfloat16*>(dst), 2 * ld, m0, M, 2 * col,
+               2 * N);
+  }
+  __device__ __forceinline__ void load_f32(float4 (&v)[4], const float* src, long long ld, long long m0, long long M,
+                                           int col, int N) const {
+    load_bf16(reinterpret_cast<uint4(&)[4]>(v), reinterpret_cast<const __nv_bfloat16*>(src), 2 * ld, m0, M, 2 * col,
+              2 * N);
+  }
+};
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
   v[0] = bf16lo(u.x); v[1] = bf16hi(u.x);
   v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
   v[4] = bf16lo(u.z); v[5] = bf16hi(u.z);
@@ -388,9 +455,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int e = warp - kGemmEpiWarp0;      // 0..7
     const int quad = warp & 3;               // TMEM lane quadrant
     const int hf = e >> 2;                   // column half of the tile
-    const int row = quad * 32 + lane;        // row of this CTA's half tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+    const StageIO io{smem_u32(smem + L::off_stg + e * L::kStgBytes), lane};
     uint32_t local = 0;
     for (long long it = pair; it < P.total_items; it += npairs, ++local) {
       const GemmItem w = gemm_item(P, it);
@@ -399,12 +466,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait_warp(&acc_full[buf], (local >> 1) & 1, ab)) break;
       tc_fence_after();
       const uint32_t tacc = tbase + buf * kGemmBN + lane_off;
-      const long long m = static_cast<long long>(w.tm) * kGemmBM + rank * kGemmHalfM + row;
-      const bool row_ok = m < q.M;
       const int n0 = w.tn * kGemmBN;
+      const long long m0 = static_cast<long long>(w.tm) * kGemmBM + rank * kGemmHalfM + quad * 32;
       if (EPI == kEpiGate) {
         // hidden units [64 hf, 64 hf + 64) of this tile: Z1 at columns c, Z3 at 128 + c
         const int hid0 = w.tn * 128 + hf * 64;
+        const int nh = q.N / 2;   // hidden units (padded) = row length of A, F1, F3
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t z1[32], z3[32];
@@ -412,48 +479,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tacc + 128 + hf * 64 + c0, z3);
           tmem_wait_ld();
           const int hid = hid0 + c0;
-          if (row_ok && hid < q.N / 2) {
+          uint4 a[4], f1[4], f3[4];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float a[8], f1[8], f3[8];
+          for (int g = 0; g < 4; ++g) {
+            float va[8], v1[8], v3[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float x1 = __uint_as_float(z1[8 * g + i]), x3 = __uint_as_float(z3[8 * g + i]);
-                const float s = gemm_sigmoid(x1);
-                const float silu = x1 * s;
-                a[i] = silu * x3;
-                f3[i] = silu;
-                f1[i] = x3 * s * (1.f + x1 * (1.f - s));
-              }
-              const long long off = m * q.ldf + hid + 8 * g;
-              store_bf16x8(reinterpret_cast<__nv_bfloat16*>(q.out) + off, a);
-              if (q.f1) store_bf16x8(q.f1 + off, f1);
-              if (q.f3) store_bf16x8(q.f3 + off, f3);
+            for (int i = 0; i < 8; ++i) {
+              const float x1 = __uint_as_float(z1[8 * g + i]), x3 = __uint_as_float(z3[8 * g + i]);
+              const float sg = gemm_sigmoid(x1);
+              const float silu = x1 * sg;
+              va[i] = silu * x3;
+              v3[i] = silu;
+              v1[i] = x3 * sg * (1.f + x1 * (1.f - sg));
             }
+            a[g] = pack_bf16x8(va);
+            f1[g] = pack_bf16x8(v1);
+            f3[g] = pack_bf16x8(v3);
           }
+          io.store_bf16(a, reinterpret_cast<__nv_bfloat16*>(q.out), q.ldf, m0, q.M, hid, nh);
+          if (q.f1) io.store_bf16(f1, q.f1, q.ldf, m0, q.M, hid, nh);
+          if (q.f3) io.store_bf16(f3, q.f3, q.ldf, m0, q.M, hid, nh);
         }
       } else if (EPI == kEpiAccF32) {
         float* out = reinterpret_cast<float*>(q.out) + static_cast<long long>(w.s) * q.split_stride;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tacc + hf * 128 + c0, r);
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tacc + hf * 128 + c0, r);
           tmem_wait_ld();
           const int col = n0 + hf * 128 + c0;
-          if (row_ok && col < q.N) {
-            float4* dst = reinterpret_cast<float4*>(out + m * q.ldo + col);
+          float4 x[4];
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              if (col + 4 * v >= q.N) break;   // N is a multiple of 4
-              float4 x = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-              if (q.accumulate) {
-                const float4 o = dst[v];
-                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
-              }
-              dst[v] = x;
+          for (int v = 0; v < 4; ++v)
+            x[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                               __uint_as_float(r[4 * v + 3]));
+          if (q.accumulate) {
+            float4 o[4];
+            io.load_f32(o, out, q.ldo, m0, q.M, col, q.N);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              x[v].x += o[v].x; x[v].y += o[v].y; x[v].z += o[v].z; x[v].w += o[v].w;
             }
           }
+          io.store_f32(x, out, q.ldo, m0, q.M, col, q.N);
         }
       } else if (EPI == kEpiL2Heads) {
         // two heads of 64 columns per half
@@ -465,34 +533,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tacc + c + 32, r1);
           tmem_wait_ld();
           const int col = n0 + c;
-          if (row_ok && col < q.N) {
-            float scale = 1.f;
-            if (col < q.norm_cols) {
-              float ss = 0.f;
+          float scale = 1.f;
+          if (col < q.norm_cols) {
+            float ss = 0.f;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float a = __uint_as_float(r0[i]), b = __uint_as_float(r1[i]);
-                ss = fmaf(a, a, ss);
-                ss = fmaf(b, b, ss);
-              }
-              scale = ss > 0.f ? rsqrtf(ss) : 0.f;
+            for (int i = 0; i < 32; ++i) {
+              const float x0 = __uint_as_float(r0[i]), x1 = __uint_as_float(r1[i]);
+              ss = fmaf(x0, x0, ss);
+              ss = fmaf(x1, x1, ss);
             }
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(q.out) + m * q.ldo + q.out_col0 + col;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float v[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[8 * g + i]) * scale;
-              store_bf16x8(dst + 8 * g, v);
-            }
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float v[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r1[8 * g + i]) * scale;
-              store_bf16x8(dst + 32 + 8 * g, v);
-            }
+            scale = ss > 0.f ? rsqrtf(ss) : 0.f;
           }
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(q.out) + q.out_col0;
+          uint4 v[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = __uint_as_float(r0[8 * g + i]) * scale;
+            v[g] = pack_bf16x8(t);
+          }
+          io.store_bf16(v, dst, q.ldo, m0, q.M, col, q.N);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = __uint_as_float(r1[8 * g + i]) * scale;
+            v[g] = pack_bf16x8(t);
+          }
+          io.store_bf16(v, dst, q.ldo, m0, q.M, col + 32, q.N);
         }
       } else {
         // kEpiStore, kEpiResidual, kEpiDz: 128 columns of this half in chunks of 32
@@ -502,35 +571,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tacc + hf * 128 + c0, r);
           tmem_wait_ld();
           const int col = n0 + hf * 128 + c0;
-          if (row_ok && col < q.N) {
+          if (EPI == kEpiDz) {
+            uint4 f1[4], f3[4];
+            io.load_bf16(f1, q.f1, q.ldf, m0, q.M, col, q.N);
+            io.load_bf16(f3, q.f3, q.ldf, m0, q.M, col, q.N);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-              if (col + 8 * g >= q.N) break;   // N is a multiple of 8
-              float v[8];
+              float a1[8], a3[8];
+              unpack_bf16x8(f1[g], a1);
+              unpack_bf16x8(f3[g], a3);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[8 * g + i]);
-              if (EPI == kEpiDz) {
-                const long long off = m * q.ldf + col + 8 * g;
-                float f1[8], f3[8], d1[8], d3[8];
-                load_bf16x8(q.f1 + off, f1);
-                load_bf16x8(q.f3 + off, f3);
+              for (int i = 0; i < 8; ++i) {
+                const float da = __uint_as_float(r[8 * g + i]);
+                a1[i] *= da;
+                a3[i] *= da;
+              }
+              f1[g] = pack_bf16x8(a1);
+              f3[g] = pack_bf16x8(a3);
+            }
+            io.store_bf16(f1, q.f1, q.ldf, m0, q.M, col, q.N);
+            io.store_bf16(f3, q.f3, q.ldf, m0, q.M, col, q.N);
+          } else {
+            float v[32];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  d1[i] = v[i] * f1[i];
-                  d3[i] = v[i] * f3[i];
-                }
-                store_bf16x8(q.f1 + off, d1);
-                store_bf16x8(q.f3 + off, d3);
-              } else {
-                if (EPI == kEpiResidual) {
-                  float rr[8];
-                  load_bf16x8(q.res + m * q.ldr + q.res_col0 + col + 8 * g, rr);
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            if (EPI == kEpiResidual) {
+              uint4 rr[4];
+              io.load_bf16(rr, q.res + q.res_col0, q.ldr, m0, q.M, col, q.N);
 #pragma unroll
-                  for (int i = 0; i < 8; ++i) v[i] -= rr[i];
-                }
-                store_bf16x8(reinterpret_cast<__nv_bfloat16*>(q.out) + m * q.ldo + q.out_col0 + col + 8 * g, v);
+              for (int g = 0; g < 4; ++g) {
+                float t[8];
+                unpack_bf16x8(rr[g], t);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * g + i] -= t[i];
               }
             }
+            uint4 o[4];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) o[g] = pack_bf16x8(v + 8 * g);
+            io.store_bf16(o, reinterpret_cast<__nv_bfloat16*>(q.out) + q.out_col0, q.ldo, m0, q.M, col, q.N);
           }
         }
       }
