@@ -147,10 +147,12 @@ int ttt_sgd_update(const ttt_dims* dims, const float* theta_in, const float* gra
  * the cubic iteration for the orthogonal polar factor is the reading taken,
  * with no momentum and no shape factor).  The step is scale-free, so the 1/n
  * of the loss does not matter.  The loss is linear in T's output, so no
- * forward pass is needed for the gradient.  Fused path only: d in
- * {16, 32, 64}, h <= 256; wide shapes return TTT_EUNSUPPORTED.  NS5 runs in
- * FP32; everything else is as in ttt_write.  Workspace: as for ttt_write /
- * ttt_layer. */
+ * forward pass is needed for the gradient.  Both head families are
+ * supported.  On the fused path NS5 runs in FP32 FMAs, one CTA per matrix; on
+ * the wide-head path (e.g. d = 1024, h = 2048) its products run on the
+ * tensor-core GEMM with each FP32 operand split into a pair of bf16 values
+ * (about 2^-16 relative per product) and FP32 accumulation.  Everything else
+ * is as in ttt_write.  Workspace: as for ttt_write / ttt_layer. */
 int ttt_write_muon(const ttt_dims* dims, const uint16_t* K, const uint16_t* V,
                    const float* conv_w, const float* theta0, float lr, int steps,
                    float* theta_out, void* workspace, size_t workspace_bytes, void* stream);
@@ -162,9 +164,11 @@ int ttt_layer_muon(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, c
 /* The Muon write sharded over processes, as ttt_grad / ttt_sgd_update are for
  * the mean-squared loss.  ttt_grad_dot: grad = d/dtheta of
  * -sum_i <T_theta(k_i), vp_i> over the tokens dims describes (workspace of
- * TTT_OP_WRITE).  ttt_muon_update: theta_out = theta_in - lr * NS5(grads[0] +
- * ... + grads[n_grads - 1]) per weight matrix of each head, the sum in index
- * order; theta_out may alias theta_in; no workspace. */
+ * TTT_OP_WRITE; both head families).  ttt_muon_update: theta_out =
+ * theta_in - lr * NS5(grads[0] + ... + grads[n_grads - 1]) per weight matrix
+ * of each head, the sum in index order; theta_out may alias theta_in; no
+ * workspace, so fused shapes only (the wide-head Newton-Schulz needs scratch
+ * for its GEMM operands; wide shapes return TTT_EUNSUPPORTED). */
 int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, const float* theta,
                  float* grad, void* workspace, size_t workspace_bytes, void* stream);
 int ttt_muon_update(const ttt_dims* dims, const float* theta_in, const float* grads, int n_grads,

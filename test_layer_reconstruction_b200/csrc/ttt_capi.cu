@@ -98,6 +98,7 @@ Grids grids_for(const Shape& s, int sms) {
 struct Ws {
   size_t status, w13, w2h, wt, vp, e, part, grad, q, k, v, o, convw, th0, thout, total;
   size_t img, img2, acc, z1, z3, ab, eb;   // wide path
+  size_t nsx, nsy, nsg, nsxh, nsxl, nsgh, nsgl, nsp;   // wide path: Newton-Schulz scratch
 };
 
 Ws ws_layout(const Shape& s, const Grids& g, int op) {
@@ -124,6 +125,17 @@ Ws ws_layout(const Shape& s, const Grids& g, int op) {
       w.eb = take(nc * s.D * 2);                                      // E = Y - V'
       w.acc = take(static_cast<size_t>(kWideMaxSplits) * 3 * s.D * s.h * 4);
       w.vp = take(tok_bytes);
+      // Muon steps: the gradient, then Newton-Schulz on one d x h matrix at a time
+      const size_t dh = static_cast<size_t>(s.D) * s.h, dd = static_cast<size_t>(s.D) * s.D;
+      w.grad = take(theta_bytes);
+      w.nsx = take(dh * 4);
+      w.nsy = take(dh * 4);
+      w.nsg = take(dd * 4);
+      w.nsxh = take(dh * 2);
+      w.nsxl = take(dh * 2);
+      w.nsgh = take(dd * 2);
+      w.nsgl = take(dd * 2);
+      w.nsp = take(kNsParts * 4);
     }
     if (op == TTT_OP_LAYER_HOST) {
       w.q = take(tok_bytes);
@@ -555,7 +567,10 @@ int wide_gate_chunk(const Call& c, const uint16_t* X, int head, long long t0, in
 //   A, F1, F3 (gate GEMM) -> E = A W2 - V' -> dA = E W2^T, dZ1 = dA F1, dZ3 = dA F3
 //   -> dW1 += K^T dZ1, dW3 += K^T dZ3, dW2 += A^T E   (FP32 split-K partials, Eq. 5)
 // into the workspace accumulator [splits][dW1 | dW3 | dW2]; returns the split count.
-int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int head, int* splits_out) {
+// With `dot` (the dot-product loss, whose output gradient is the constant
+// -V'/n) the residual GEMM is skipped and V' itself stands where E stands;
+// the caller negates.
+int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int head, int* splits_out, bool dot = false) {
   const Shape& s = c.s;
   const WideOperands w = wide_head(c, head);
   unsigned int* status = reinterpret_cast<unsigned int*>(c.ws + c.w.status);
@@ -569,7 +584,11 @@ int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int hea
   for (long long t0 = 0; t0 < s.n; t0 += kWideChunk) {
     const int nc = static_cast<int>(std::min<long long>(kWideChunk, s.n - t0));
     if ((rc = wide_gate_chunk(c, K, head, t0, nc, true)) != TTT_OK) return rc;
-    {  // E = A W2 - V'
+    // E: [nc][d] in the chunk buffer (pitch d), or V' in place (pitch C, the head's columns)
+    const __nv_bfloat16* e_src = dot ? reinterpret_cast<const __nv_bfloat16*>(vp) + static_cast<size_t>(t0) * s.C : eb;
+    const long long e_pitch = dot ? s.C : s.D, e_cols = dot ? s.C : s.D;
+    const int e_x0 = dot ? head * s.D : 0;
+    if (!dot) {  // E = A W2 - V'
       GemmLaunch g;
       if (!make_gemm_map(&g.ma[0], ab, nc, s.hidp, s.hidp, false) ||
           !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, true))
@@ -584,9 +603,11 @@ int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int hea
     }
     {  // dA = E W2^T, then dZ1 = dA F1, dZ3 = dA F3 in place
       GemmLaunch g;
-      if (!make_gemm_map(&g.ma[0], eb, nc, s.D, s.D, false) || !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, false))
+      if (!make_gemm_map(&g.ma[0], e_src, nc, e_cols, e_pitch, false) ||
+          !make_gemm_map(&g.mb[0], w.img2, s.h, s.D, s.D, false))
         return TTT_ECUDA;
       GemmProblem& q = g.add(nc, s.hidp, s.D, false, false);
+      q.a_x0 = e_x0;
       q.f1 = f1;
       q.f3 = f3;
       q.ldf = s.hidp;
@@ -597,7 +618,8 @@ int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int hea
       const uint16_t* kc = K + static_cast<size_t>(t0) * s.C;
       if (!make_gemm_map(&g.ma[0], kc, nc, s.C, s.C, true) || !make_gemm_map(&g.mb[0], f1, nc, s.hidp, s.hidp, true) ||
           !make_gemm_map(&g.ma[1], kc, nc, s.C, s.C, true) || !make_gemm_map(&g.mb[1], f3, nc, s.hidp, s.hidp, true) ||
-          !make_gemm_map(&g.ma[2], ab, nc, s.hidp, s.hidp, true) || !make_gemm_map(&g.mb[2], eb, nc, s.D, s.D, true))
+          !make_gemm_map(&g.ma[2], ab, nc, s.hidp, s.hidp, true) ||
+          !make_gemm_map(&g.mb[2], e_src, nc, e_cols, e_pitch, true))
         return TTT_ECUDA;
       // The first chunk is the largest and fixes the split count: every later
       // chunk adds its split s into partial s (it may have fewer splits,
@@ -611,6 +633,7 @@ int wide_grad_head(const Call& c, const uint16_t* K, const uint16_t* vp, int hea
       for (int m = 0; m < 3; ++m) {
         GemmProblem& q = *qs[m];
         q.a_x0 = m < 2 ? head * s.D : 0;
+        if (m == 2) q.b_x0 = e_x0;
         q.out = acc + m * per;
         q.ldo = m < 2 ? s.h : s.D;
         q.split_stride = 3 * per;
@@ -655,8 +678,10 @@ int run_write_wide(const Call& c, const ttt_dims* dm, const uint16_t* K, const u
   return TTT_OK;
 }
 
-// The gradient (1/2) d/dtheta sum_i ||T(k_i) - v'_i||^2 of the wide path.
-int run_grad_wide(const Call& c, const uint16_t* K, const uint16_t* vp, const float* theta, float* grad) {
+// The gradient (1/2) d/dtheta sum_i ||T(k_i) - v'_i||^2 of the wide path, or
+// with `dot` that of -sum_i <T(k_i), v'_i>.
+int run_grad_wide(const Call& c, const uint16_t* K, const uint16_t* vp, const float* theta, float* grad,
+                  bool dot = false) {
   const Shape& s = c.s;
   const long long per = static_cast<long long>(s.D) * s.h;
   const float* acc = reinterpret_cast<const float*>(c.ws + c.w.acc);
@@ -664,10 +689,82 @@ int run_grad_wide(const Call& c, const uint16_t* K, const uint16_t* vp, const fl
   if (rc != TTT_OK) return rc;
   for (int head = 0; head < s.H; ++head) {
     int splits = 1;
-    if ((rc = wide_grad_head(c, K, vp, head, &splits)) != TTT_OK) return rc;
+    if ((rc = wide_grad_head(c, K, vp, head, &splits, dot)) != TTT_OK) return rc;
     ProfScope prof(KK_REDUCE, c.st);
-    wide_grad_kernel<<<elementwise_grid(3 * per), 256, 0, c.st>>>(grad, acc, splits, s.H, s.D, s.h, head);
+    wide_grad_kernel<<<elementwise_grid(3 * per), 256, 0, c.st>>>(grad, acc, splits, s.H, s.D, s.h, head,
+                                                                   dot ? -1.f : 1.f);
     if ((rc = launch_status()) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
+// out (f32 [M][N], row pitch ldo) = or += A B on the tensor-core GEMM, A and B
+// bf16 in the given layouts (A: [M][K] K-major or [K][M]; B: [N][K] K-major
+// or [K][N]).
+int gemm_f32(const Call& c, const __nv_bfloat16* A, bool a_mn, const __nv_bfloat16* B, bool b_mn, int M, int N, int K,
+             float* out, long long ldo, bool accumulate) {
+  GemmLaunch g;
+  if (!make_gemm_map(&g.ma[0], A, a_mn ? K : M, a_mn ? M : K, a_mn ? M : K, a_mn) ||
+      !make_gemm_map(&g.mb[0], B, b_mn ? K : N, b_mn ? N : K, b_mn ? N : K, b_mn))
+    return TTT_ECUDA;
+  GemmProblem& q = g.add(M, N, K, a_mn, b_mn);
+  q.out = out;
+  q.ldo = ldo;
+  q.accumulate = accumulate ? 1 : 0;
+  return launch_gemm<kEpiAccF32>(g, reinterpret_cast<unsigned int*>(c.ws + c.w.status), KK_REDUCE, c.st);
+}
+
+// theta_out = theta_in - lr NS5(sum of n_grads gradients) on the wide path,
+// per head and matrix (reading 10; products split into bf16 pairs, wide.cuh).
+int run_muon_update_wide(const Call& c, const float* theta_in, const float* grads, int n_grads, float lr,
+                         float* theta_out) {
+  const Shape& s = c.s;
+  const int d = s.D, h = s.h;
+  const long long dh = static_cast<long long>(d) * h, dd = static_cast<long long>(d) * d;
+  float* X = reinterpret_cast<float*>(c.ws + c.w.nsx);
+  float* Y = reinterpret_cast<float*>(c.ws + c.w.nsy);
+  float* G = reinterpret_cast<float*>(c.ws + c.w.nsg);
+  __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.nsxh);
+  __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.nsxl);
+  __nv_bfloat16* gh = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.nsgh);
+  __nv_bfloat16* gl = reinterpret_cast<__nv_bfloat16*>(c.ws + c.w.nsgl);
+  float* part = reinterpret_cast<float*>(c.ws + c.w.nsp);
+  int rc;
+  for (int head = 0; head < s.H; ++head) {
+    for (int m = 0; m < 3; ++m) {
+      {
+        ProfScope prof(KK_REDUCE, c.st);
+        ns_load_kernel<<<kNsParts, 256, 0, c.st>>>(grads, n_grads, s.H, d, h, head, m, X, part);
+        ns_normalise_kernel<<<elementwise_grid(dh), 256, 0, c.st>>>(X, part, dh, xh, xl);
+      }
+      if ((rc = launch_status()) != TTT_OK) return rc;
+      for (int it = 0; it < kNsIters; ++it) {
+        // Gram = X X^T (B = X read K-major), split; Y = Gram X (B = X read MN-major)
+        if ((rc = gemm_f32(c, xh, false, xh, false, d, d, h, G, d, false)) != TTT_OK ||
+            (rc = gemm_f32(c, xh, false, xl, false, d, d, h, G, d, true)) != TTT_OK ||
+            (rc = gemm_f32(c, xl, false, xh, false, d, d, h, G, d, true)) != TTT_OK)
+          return rc;
+        {
+          ProfScope prof(KK_REDUCE, c.st);
+          ns_split_kernel<<<elementwise_grid(dd), 256, 0, c.st>>>(G, dd, gh, gl);
+        }
+        if ((rc = launch_status()) != TTT_OK) return rc;
+        if ((rc = gemm_f32(c, gh, false, xh, true, d, h, d, Y, h, false)) != TTT_OK ||
+            (rc = gemm_f32(c, gh, false, xl, true, d, h, d, Y, h, true)) != TTT_OK ||
+            (rc = gemm_f32(c, gl, false, xh, true, d, h, d, Y, h, true)) != TTT_OK)
+          return rc;
+        {
+          ProfScope prof(KK_REDUCE, c.st);
+          ns_combine_kernel<<<elementwise_grid(dh), 256, 0, c.st>>>(X, Y, dh, xh, xl);
+        }
+        if ((rc = launch_status()) != TTT_OK) return rc;
+      }
+      {
+        ProfScope prof(KK_REDUCE, c.st);
+        ns_apply_kernel<<<elementwise_grid(dh), 256, 0, c.st>>>(theta_in, theta_out, X, s.H, d, h, head, m, lr);
+      }
+      if ((rc = launch_status()) != TTT_OK) return rc;
+    }
   }
   return TTT_OK;
 }
@@ -823,12 +920,21 @@ int run_write_muon(const Call& c, const ttt_dims* dm, const uint16_t* K, const u
   const Shape& s = c.s;
   uint16_t* vp = reinterpret_cast<uint16_t*>(c.ws + c.w.vp);
   float* grad = reinterpret_cast<float*>(c.ws + c.w.grad);
-  int rc = run_conv(s, dm, V, conv_w, vp, c.st, true);
+  // the wide path's GEMMs read V' in bf16; the fused backward in f16
+  int rc = run_conv(s, dm, V, conv_w, vp, c.st, !s.wide);
   if (rc != TTT_OK) return rc;
   if (steps == 0) {
     if (theta_out != theta0 &&
         cudaMemcpyAsync(theta_out, theta0, 3ull * s.H * s.D * s.h * 4, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
       return TTT_ECUDA;
+    return TTT_OK;
+  }
+  if (s.wide) {
+    for (int step = 0; step < steps; ++step) {
+      const float* th_in = step == 0 ? theta0 : theta_out;
+      if ((rc = run_grad_wide(c, K, vp, th_in, grad, true)) != TTT_OK) return rc;
+      if ((rc = run_muon_update_wide(c, th_in, grad, 1, lr, theta_out)) != TTT_OK) return rc;
+    }
     return TTT_OK;
   }
   GradPass gp;
@@ -1026,11 +1132,10 @@ int ttt_grad_dot(const ttt_dims* dims, const uint16_t* K, const uint16_t* Vp, co
                  void* workspace, size_t workspace_bytes, void* stream) {
   if (!K || !Vp || !theta || !grad) return TTT_EINVAL;
   if (!aligned(K) || !aligned(Vp) || !aligned(theta) || !aligned(grad)) return TTT_EALIGN;
-  int rc = fused_only(dims);
-  if (rc != TTT_OK) return rc;
   Call c;
-  rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
+  if (c.s.wide) return run_grad_wide(c, K, Vp, theta, grad, true);
   // the backward kernel reads V' in f16, its operand type
   uint16_t* vp16 = reinterpret_cast<uint16_t*>(c.ws + c.w.e);
   const long long count = c.s.n * c.s.C;
@@ -1058,10 +1163,8 @@ int ttt_write_muon(const ttt_dims* dims, const uint16_t* K, const uint16_t* V, c
                    size_t workspace_bytes, void* stream) {
   if (!K || !V || !conv_w || !theta0 || !theta_out || steps < 0) return TTT_EINVAL;
   if (!aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out)) return TTT_EALIGN;
-  int rc = fused_only(dims);
-  if (rc != TTT_OK) return rc;
   Call c;
-  rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
+  int rc = prepare(dims, TTT_OP_WRITE, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
   return run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out);
 }
@@ -1073,10 +1176,8 @@ int ttt_layer_muon(const ttt_dims* dims, const uint16_t* Q, const uint16_t* K, c
   if (!aligned(Q) || !aligned(K) || !aligned(V) || !aligned(conv_w) || !aligned(theta0) || !aligned(theta_out) ||
       !aligned(O))
     return TTT_EALIGN;
-  int rc = fused_only(dims);
-  if (rc != TTT_OK) return rc;
   Call c;
-  rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
+  int rc = prepare(dims, TTT_OP_LAYER, workspace, workspace_bytes, stream, &c);
   if (rc != TTT_OK) return rc;
   if ((rc = run_write_muon(c, dims, K, V, conv_w, theta0, lr, steps, theta_out)) != TTT_OK) return rc;
   return run_read(c, Q, theta_out, O);

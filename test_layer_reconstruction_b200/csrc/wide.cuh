@@ -15,6 +15,7 @@
 //   wide_sgd_kernel   theta_out = theta_in - scale * (sum of the split-K
 //                     partials of dW, in split order) for one head
 //   wide_grad_kernel  the same sum written into a gradient in theta's layout
+//   ns_*_kernel       the elementwise steps of Newton-Schulz (Muon) on wide heads
 #pragma once
 #include "sm100.cuh"
 
@@ -59,16 +60,118 @@ __global__ void wide_sgd_kernel(const float* theta_in, float* theta_out, const f
   }
 }
 
-// grad = sum_{s < splits} dw[s] of head `head`, scattered into theta's per-head layout.
+// grad = sign * sum_{s < splits} dw[s] of head `head`, scattered into theta's per-head layout.
 __global__ void wide_grad_kernel(float* grad, const float* __restrict__ dw, int splits, int heads, int d, int h,
-                                 int head) {
+                                 int head, float sign) {
   const long long per = static_cast<long long>(d) * h;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < 3 * per;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     float g = dw[e];
     for (int s = 1; s < splits; ++s) g += dw[s * 3 * per + e];
     const long long m = e / per, r = e % per;
-    grad[m * heads * per + static_cast<long long>(head) * per + r] = g;
+    grad[m * heads * per + static_cast<long long>(head) * per + r] = sign * g;
+  }
+}
+
+// ------------------------------------------------------------------ Muon on wide heads
+// The pages' inner optimiser (Sec. 3.4, "TTT MLP Architecture and Inner
+// Optimization": Muon, 5 Newton-Schulz iterations) for heads whose matrices
+// no longer fit one CTA: per weight matrix, X_0 = G / ||G||_F, then
+// X <- 1.5 X - 0.5 (X X^T) X five times, theta <- theta - lr X_5, with W2's
+// h x d gradient transposed to d x h (the iteration commutes with
+// transposition).  The products run on the tensor-core GEMM with FP32
+// operands split into bf16 pairs, hi = bf16(x), lo = bf16(x - hi), and
+// x y = hi_x hi_y + hi_x lo_y + lo_x hi_y (the lo_x lo_y term, ~2^-16 of the
+// product, is dropped), accumulated in FP32: the splitting scheme of Henry,
+// Tang and Heinecke (using bfloat16 for higher-precision computation, ARITH
+// 2019), about 2^-16 relative per product instead of bf16's 2^-8.  Sums of
+// squares are reduced in a fixed order, so the step is deterministic.
+constexpr int kNsParts = 256;   // blocks of the norm reduction
+
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  *hi = h;
+  *lo = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
+// X [d][h] = sum_r grads[r] of matrix m of head `head` (W2 transposed), and
+// per-block partial sums of squares.  Launched with kNsParts blocks.
+__global__ void ns_load_kernel(const float* __restrict__ grads, int n_grads, int heads, int d, int h, int head,
+                               int m, float* __restrict__ X, float* __restrict__ partial) {
+  const long long per = static_cast<long long>(d) * h;
+  const long long count = 3LL * heads * per;
+  const long long base = m * heads * per + static_cast<long long>(head) * per;
+  float ss = 0.f;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < per;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = e / h, c = e % h;   // X[i][c]
+    const long long o = base + (m < 2 ? i * h + c : c * d + i);
+    float g = grads[o];
+    for (int r = 1; r < n_grads; ++r) g += grads[static_cast<long long>(r) * count + o];
+    X[e] = g;
+    ss = fmaf(g, g, ss);
+  }
+  __shared__ float red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += red[w];
+    partial[blockIdx.x] = t;
+  }
+}
+
+// X *= 1 / ||X||_F (the partial sums added in block order; a zero matrix stays
+// zero), then the bf16 pair of X.
+__global__ void ns_normalise_kernel(float* __restrict__ X, const float* __restrict__ partial, long long count,
+                                    __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  __shared__ float inv;
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int b = 0; b < kNsParts; ++b) t += partial[b];
+    inv = t > 0.f ? 1.f / sqrtf(t) : 0.f;
+  }
+  __syncthreads();
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float x = X[e] * inv;
+    X[e] = x;
+    split_bf16(x, hi + e, lo + e);
+  }
+}
+
+// The bf16 pair of an FP32 matrix.
+__global__ void ns_split_kernel(const float* __restrict__ G, long long count, __nv_bfloat16* __restrict__ hi,
+                                __nv_bfloat16* __restrict__ lo) {
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
+       e += static_cast<long long>(gridDim.x) * blockDim.x)
+    split_bf16(G[e], hi + e, lo + e);
+}
+
+// X <- 1.5 X - 0.5 Y, Y = (X X^T) X; then the bf16 pair of X.
+__global__ void ns_combine_kernel(float* __restrict__ X, const float* __restrict__ Y, long long count,
+                                  __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float x = 1.5f * X[e] - 0.5f * Y[e];
+    X[e] = x;
+    split_bf16(x, hi + e, lo + e);
+  }
+}
+
+// theta_out = theta_in - lr X for matrix m of head `head` (W2 transposed back).
+// theta_out may alias theta_in.
+__global__ void ns_apply_kernel(const float* theta_in, float* theta_out, const float* __restrict__ X, int heads,
+                                int d, int h, int head, int m, float lr) {
+  const long long per = static_cast<long long>(d) * h;
+  const long long base = m * heads * per + static_cast<long long>(head) * per;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < per;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = e / h, c = e % h;
+    const long long o = base + (m < 2 ? i * h + c : c * d + i);
+    theta_out[o] = theta_in[o] - lr * X[e];
   }
 }
 

@@ -122,3 +122,59 @@ def test_muon_write_equals_its_pieces_bitwise():
     torch.cuda.synchronize()
     assert torch.equal(full, pieces)
     assert torch.equal(zero, dev["theta"])
+
+
+# The wide-head path (d, h multiples of 64 beyond the fused kernels): the
+# gradient on the tensor-core GEMM with V' in place of the residual, and
+# Newton-Schulz on the GEMM with each FP32 operand split into a bf16 pair
+# (about 2^-16 relative per product), FP32 accumulation.
+WIDE_CASES = [tin.LayerConfig("muon_wide_small", 3, 9, 10, 2, 2, 128, 192, 2, LR, 51),
+              tin.CONFIGS["views2000_37x37p5_h1_d1024_h2048"].with_views(4)]
+
+
+@pytest.mark.parametrize("cfg", WIDE_CASES, ids=["d128_h192", "d1024_h2048"])
+def test_wide_layer_muon_matches_oracle(cfg):
+    inp, dev = _device(cfg)
+    theta, O = ttt.layer_muon(dev["Q"], dev["K"], dev["V"], dev["conv_w"], dev["theta"], LR, 2, cfg)
+    torch.cuda.synchronize()
+    W = [t.double().numpy() for t in tin.unpack_theta(theta.cpu(), cfg.heads, cfg.d, cfg.h)]
+    Og = O.double().cpu().numpy()
+    worst_d, worst_o = 0.0, 0.0
+    for hd, (th0, th_ref, O_ref) in _oracle_muon(cfg, inp, 2, list(range(cfg.heads))).items():
+        for m in range(3):
+            worst_d = max(worst_d, normwise(W[m][hd] - th0[m], th_ref[m] - th0[m]))
+        worst_o = max(worst_o, normwise(Og[:, hd], O_ref))
+    report(f"muon_wide_{cfg.d}_{cfg.h}", delta=worst_d, O=worst_o)
+    assert worst_d <= TOL_MUON_DELTA, worst_d
+    assert worst_o <= TOL_O, worst_o
+
+
+def test_wide_grad_dot_matches_oracle():
+    cfg = WIDE_CASES[0]
+    inp, dev = _device(cfg)
+    Vp = ttt.shortconv2d(dev["V"], dev["conv_w"], cfg)
+    g = ttt.grad_dot(dev["K"], Vp, dev["theta"], cfg)
+    torch.cuda.synchronize()
+    G = [t.double().numpy() for t in tin.unpack_theta(g.cpu(), cfg.heads, cfg.d, cfg.h)]
+    dims = dims_of(cfg)
+    n, H, d = inp["K"].shape
+    worst = 0.0
+    for hd in range(H):
+        ch = slice(hd * d, (hd + 1) * d)
+        vp = orc.shortconv2d(inp["V"][:, hd].double().numpy(), inp["conv_w"][ch].double().numpy(), dims)
+        ref = orc.dot_grad(inp["K"][:, hd].double().numpy(), vp, inp["W1"][hd].double().numpy(),
+                           inp["W3"][hd].double().numpy(), inp["W2"][hd].double().numpy())
+        worst = max(worst, *(normwise(G[m][hd], ref[m] * n) for m in range(3)))
+    report("muon_wide_grad_dot", grad=worst)
+    assert worst <= TOL_DELTA, worst
+
+
+def test_wide_muon_write_is_deterministic_and_lr0_keeps_theta():
+    cfg = WIDE_CASES[0]
+    _, dev = _device(cfg)
+    a = ttt.write_muon(dev["K"], dev["V"], dev["conv_w"], dev["theta"], LR, 2, cfg)
+    b = ttt.write_muon(dev["K"], dev["V"], dev["conv_w"], dev["theta"], LR, 2, cfg)
+    z = ttt.write_muon(dev["K"], dev["V"], dev["conv_w"], dev["theta"], 0.0, 2, cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(z, dev["theta"])
