@@ -18,10 +18,10 @@
 //              chunks c with c % 2 == p, one 32-unit half of the chunk each
 // Both issuers run in uniform control flow and issue from one elected lane.
 // Per tile the hidden dimension is walked in chunks of 64 units:
-//   Z = X * [W1 | W3]_chunk        (M=128 tokens, N=128, K=d, A and B in smem)
+//   Z = X * [W1/2 | W3]_chunk      (M=128 tokens, N=128, K=d, A and B in smem)
 //                                    -> TMEM Z slot c % 2
 //   gate = silu(Z1) * Z3           (epilogue warpgroups 2(c%2), 2(c%2)+1, packed
-//                                    f16 arithmetic) -> TMEM gate slot c % 2
+//                                    f16 arithmetic on Z1/2) -> TMEM gate slot c % 2
 //   Y += gate * W2_chunk           (M=128, N=d, K=64, A from TMEM, B = f16 W2
 //                                    image in smem) -> TMEM Y slot j % 2
 // Keeping the gate in tensor memory avoids a shared-memory round trip and
@@ -117,14 +117,14 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Gate of two hidden units in packed f16: silu(z1) * z3 with
-// sigmoid(z) = (1 + tanh(z/2)) / 2.
-__device__ __forceinline__ uint32_t gate_f16x2(float z1a, float z1b, float z3a, float z3b) {
-  const uint32_t h1 = pack_f16x2(z1a, z1b);
+// Gate of two hidden units in packed f16: silu(z1) * z3.  The Z1 columns
+// hold u = z1/2 (the W1 operand image is halved, exactly), and with
+// t = tanh(u): sigmoid(z1) = (1 + t)/2, so silu(z1) = u (1 + t) = u + u t.
+__device__ __forceinline__ uint32_t gate_f16x2(float ua, float ub, float z3a, float z3b) {
+  const uint32_t hu = pack_f16x2(ua, ub);
   const uint32_t h3 = pack_f16x2(z3a, z3b);
-  const uint32_t t = htanh2(hmul2(h1, kHalf2Half));
-  const uint32_t s = hfma2(t, kHalf2Half, kHalf2Half);
-  return hmul2(hmul2(h1, s), h3);
+  const uint32_t t = htanh2(hu);
+  return hmul2(hfma2(hu, t, hu), h3);
 }
 
 template <int D, int HIDP, bool WRITE>

@@ -20,7 +20,8 @@
 // units padded with zeros up to HIDP:
 //   W13 image (bf16), per head, laid out as the forward kernel's shared-memory
 //     tile (rows of D elements, swizzled by 8-row atoms): for every 32-unit
-//     sub-chunk s, 32 rows of W1^T (hidden s*32+r) then 32 rows of W3^T.
+//     sub-chunk s, 32 rows of W1^T / 2 (hidden s*32+r; halving is exact) then
+//     32 rows of W3^T.
 //   W2 image (f16, same tiling), per head: row j = W2[j][:]; the forward
 //     kernel's gate operand is f16.
 //   WT image (f16, plain rows; write path only), per head and hidden unit r:
@@ -122,6 +123,7 @@ __global__ void pack_images_kernel(const PackParams p) {
     if (hid < p.h) {
       const float* w = p.theta + (rr < 32 ? 0 : hdh);
       v = w[static_cast<size_t>(head) * D * p.h + static_cast<size_t>(col) * p.h + hid];
+      if (rr < 32) v *= 0.5f;   // W1 halved (exact): the forward gate reads u = z1/2
     }
     const uint32_t off = swz(static_cast<uint32_t>(R) * SW + col * 2, SW);
     *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(p.w13_img + static_cast<size_t>(head) * 2 * p.hidp * D) + off) =
