@@ -12,7 +12,8 @@
 //   dW1^T += dZ1^T K,  dW3^T += dZ3^T K,  dW2 += A^T E
 //
 // Hidden-major formulation.  All products are taken with the hidden units on
-// the 128 TMEM lanes (M=128 hidden, N=48 tokens, K=d):
+// the 128 TMEM lanes (M=128 hidden, N=48 tokens, K=d; f16 operands, FP32
+// accumulators):
 //   U^T = (W1/2)^T K^T   A = the slice's W1^T/2 rows kept in TMEM (TS)
 //   Z3^T = W3^T K^T      A = the slice's W3^T rows in shared memory (SS)
 //   dA^T = W2 E^T        A = the slice's W2 rows in shared memory (SS)
@@ -38,8 +39,9 @@
 // partials of a (head, slice) in group order, so the result is deterministic.
 //
 // Warp roles: warp 0 TMA producer; warp 1 TMEM allocator and U/Z3/dA issuer;
-// warp 2 dW issuer; warp 3 idle; warps 4-15 three epilogue warpgroups, group g
-// owning tokens 16g..16g+15 of every unit.  Both issuers run warp-uniform loops
+// warp 2 dW issuer; warp 3 converts each landed K tile to f16 in place; warps
+// 4-15 three epilogue warpgroups, group g owning tokens 16g..16g+15 of every
+// unit.  Both issuers run warp-uniform loops
 // with precomputed descriptors and issue from one elected lane.
 #pragma once
 #include "fwd.cuh"
