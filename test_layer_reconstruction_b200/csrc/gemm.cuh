@@ -226,7 +226,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-__device__ __forceinline__ float gemm_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+// One MUFU operation per element: sigmoid(z) = (1 + tanh(z/2)) / 2.
+__device__ __forceinline__ float gemm_sigmoid(float z) { return sigmoid_fast(z); }
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
   uint4 u;
