@@ -21,7 +21,8 @@
 //   Z = X * [W1/2 | W3]_chunk      (M=128 tokens, N=128, K=d, A and B in smem)
 //                                    -> TMEM Z slot c % 2
 //   gate = silu(Z1) * Z3           (epilogue warpgroups 2(c%2), 2(c%2)+1, packed
-//                                    f16 arithmetic on Z1/2) -> TMEM gate slot c % 2
+//                                    f16 arithmetic on Z1/2) -> TMEM gate slot
+//                                    (three, taken in turn by every chunk of every tile)
 //   Y += gate * W2_chunk           (M=128, N=d, K=64, A from TMEM, B = f16 W2
 //                                    image in smem) -> TMEM Y slot j % 2
 // Keeping the gate in tensor memory avoids a shared-memory round trip and
@@ -59,21 +60,22 @@ struct FwdLayout {
   static constexpr uint32_t off_x = off_w2 + kW2;
   static constexpr uint32_t off_vp = off_x + 2 * kTile;
   static constexpr uint32_t off_bar = off_vp + 2 * kTile;
-  static constexpr int kNumBars = 24;
+  static constexpr int kNumBars = 30;
   static constexpr uint32_t bytes = off_bar + kNumBars * 8 + 16 + 1024;
   static_assert(off_x % 1024 == 0 && off_vp % 1024 == 0, "1 KiB alignment");
 };
 
 // TMEM columns
 constexpr uint32_t kFwdZCols = 0;      // 2 Z slots x 128
-constexpr uint32_t kFwdGateCols = 256; // 2 gate slots x 32 (64 f16 per row)
-constexpr uint32_t kFwdYCols = 320;    // 2 Y slots x D
+constexpr uint32_t kFwdGateCols = 256; // kFwdGateSlots gate slots x 32 (64 f16 per row)
+constexpr int kFwdGateSlots = 3;       // taken in turn by the chunks of all tiles
+constexpr uint32_t kFwdYCols = 352;    // 2 Y slots x D
 
 // barrier indices
 enum FwdBar {
   FB_W_FULL = 0, FB_W_EMPTY = 1, FB_X_FULL = 2, FB_X_EMPTY = 4, FB_VP_FULL = 6, FB_VP_EMPTY = 8,
-  FB_Z_FULL = 10, FB_Z_EMPTY = 12, FB_A_FULL = 14, FB_A_EMPTY = 16, FB_Y_FULL = 18, FB_Y_EMPTY = 20,
-  FB_DONE = 22
+  FB_Z_FULL = 10, FB_Z_EMPTY = 12, FB_Y_FULL = 18, FB_Y_EMPTY = 20,
+  FB_DONE = 22, FB_G_FULL = 24, FB_G_EMPTY = FB_G_FULL + kFwdGateSlots
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -158,10 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[FB_VP_EMPTY + s], 8);
       mbar_init(&bars[FB_Z_FULL + s], 1);
       mbar_init(&bars[FB_Z_EMPTY + s], 8);
-      mbar_init(&bars[FB_A_FULL + s], 8);
-      mbar_init(&bars[FB_A_EMPTY + s], 1);
       mbar_init(&bars[FB_Y_FULL + s], 1);
       mbar_init(&bars[FB_Y_EMPTY + s], 8);
+    }
+    for (int s = 0; s < kFwdGateSlots; ++s) {
+      mbar_init(&bars[FB_G_FULL + s], 8);    // the eight warps of the pair that gated the chunk
+      mbar_init(&bars[FB_G_EMPTY + s], 1);
     }
     mbar_init(&bars[FB_DONE], 2);
     fence_mbar_init();
@@ -303,16 +307,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ys = yj & 1;
       if (!(ok = mbar_wait_warp(&bars[FB_Y_EMPTY + ys], ((yj >> 1) & 1) ^ 1, ab))) break;
       for (int c = 0; c < NC; ++c) {
-        const int g = c & 1;
-        const uint32_t u = yj * (NC / 2) + (c >> 1);
-        if (!(ok = mbar_wait_warp(&bars[FB_A_FULL + g], u & 1, ab))) break;
+        const uint32_t gc = yj * NC + c;   // chunk counter: gate slot gc % kFwdGateSlots
+        const uint32_t gs = gc % kFwdGateSlots;
+        if (!(ok = mbar_wait_warp(&bars[FB_G_FULL + gs], (gc / kFwdGateSlots) & 1, ab))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint64_t bd = smem_desc(w2 + (64 * c + 16 * k) * SW, HIDP * SW, 8 * SW, SW);
-          mma_bf16_ts_warp(ty + ys * D, tg + g * 32 + 8 * k, bd, kIdY, (c > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ts_warp(ty + ys * D, tg + gs * 32 + 8 * k, bd, kIdY, (c > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit_warp(&bars[FB_A_EMPTY + g]);
+        mma_commit_warp(&bars[FB_G_EMPTY + gs]);
       }
       if (ok) mma_commit_warp(&bars[FB_Y_FULL + ys]);
     }
@@ -430,14 +434,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[FB_Z_EMPTY + pr]);
         TTT_TR_LAP(2);
-        if (!(ok = mbar_wait_warp(&bars[FB_A_EMPTY + pr], (u & 1) ^ 1, ab))) break;
+        const uint32_t gc = j * NC + c;   // chunk counter: gate slot gc % kFwdGateSlots
+        const uint32_t gs = gc % kFwdGateSlots;
+        if (!(ok = mbar_wait_warp(&bars[FB_G_EMPTY + gs], ((gc / kFwdGateSlots) & 1) ^ 1, ab))) break;
         TTT_TR_LAP(3);
         tc_fence_after();
-        tmem_st16(tg + pr * 32 + hf * 16 + lane_off, gk);
+        tmem_st16(tg + gs * 32 + hf * 16 + lane_off, gk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[FB_A_FULL + pr]);
+        if (lane == 0) mbar_arrive(&bars[FB_G_FULL + gs]);
         TTT_TR_LAP(4);
       }
       if (!ok) break;
